@@ -1,0 +1,165 @@
+"""Plain fp64 CPU oracle for the high-rank DoRA hot path.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports this module:
+only the tests, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` may call it.  It shares no code with
+the CUDA library (no kernels, headers, helpers or constants); both sides only
+consume the same seeded inputs.
+
+What it computes, and where that is defined
+-------------------------------------------
+Sources are the pages this project was specified from:
+
+* "Scaling DoRA: High-Rank Adaptation via Factored Norms and Fused Kernels"
+  (Zelenin & Zhuravlyova, arXiv 2603.22276), Abstract: DoRA's forward pass
+  needs the row-wise norm of ``W + sBA``; frameworks materialise the dense
+  ``[d_out, d_in]`` product ``BA`` to get it; the magnitude rescaling is then
+  composed with the base and LoRA outputs.
+* "DoRA: Weight-decomposed low-rank adaptation" (summary page, section
+  "Method"): the pretrained weight is split into a magnitude vector and a
+  direction matrix normalised per output channel; the low-rank update adapts
+  the direction only.
+
+The factored norm of the first page reaches *exactly* (up to rounding order)
+the dense row norm, so this oracle is the plain definition written out, not
+the factored algorithm:
+
+    W' = W + s * (B @ A)                  dense [d_out, d_in], fp64
+    n_i = sqrt(sum_k W'_ik ** 2)          one norm per output channel
+    g_i = m_i / n_i
+    y[t, i] = g_i * (base[t, i] + s * lora[t, i])
+
+Backward (the norm ``n`` is held constant, see ``compose_backward``) with an
+upstream gradient ``dy``:
+
+    d_base = g * dy
+    d_lora = s * g * dy
+    d_m_i  = sum_t dy[t, i] * (base[t, i] + s * lora[t, i]) / n_i
+
+Layout convention (PyTorch ``nn.Linear``): ``W`` is ``[d_out, d_in]``, ``A``
+(lora_A) is ``[r, d_in]``, ``B`` (lora_B) is ``[d_out, r]``; activations are
+``[tokens, d_out]`` row-major; ``m``/``n`` are per output channel.  The
+"column-wise" norm of the DoRA summary page is written for a ``[d, k]`` weight
+whose columns are output channels; in ``[d_out, d_in]`` storage the same norm
+is taken along each row.
+
+Readings where the pages are silent (each also listed in the design notes):
+
+* ``n`` is detached in backward (no gradient flows into ``A``/``B`` through
+  the norm).  The DoRA summary page ("Statistical analysis" / "Strengths")
+  mentions a training-memory modification of the original method; treating
+  the norm as a constant is the plainest reading consistent with the three
+  outputs the hot path is asked for.
+* No epsilon is invented: ``n_i^2`` is used as computed; ``n_i == 0`` gives
+  IEEE inf/nan in ``g`` exactly as the definition does.
+* No bias term: ``base`` is bias-free.
+
+Every function takes float64 numpy arrays (callers round bf16 inputs first,
+then widen) and returns float64 results.  No blocking, fusion or reordering
+beyond what the definition states.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "dense_adapted_weight",
+    "row_norm",
+    "row_norm_rows",
+    "magnitude_scale",
+    "compose_forward",
+    "compose_backward",
+    "compose_backward_columns",
+]
+
+
+def _f64(x) -> np.ndarray:
+    return np.asarray(x, dtype=np.float64)
+
+
+def dense_adapted_weight(W, A, B, s) -> np.ndarray:
+    """``W + s * (B @ A)``, the dense ``[d_out, d_in]`` adapted weight.
+
+    Scaling DoRA, Abstract: the product ``BA`` that every surveyed framework
+    materialises.  The oracle materialises it on purpose.
+    """
+    W, A, B = _f64(W), _f64(A), _f64(B)
+    return W + float(s) * (B @ A)
+
+
+def row_norm(W, A, B, s) -> np.ndarray:
+    """``n_i = ||W_i + s * B_i A||_2`` for every output channel i.
+
+    Scaling DoRA, Abstract ("the row-wise norm of W + sBA"); DoRA summary
+    page, Method (per-output-channel vector norm of the adapted weight).
+    """
+    Wp = dense_adapted_weight(W, A, B, s)
+    return np.sqrt(np.sum(Wp * Wp, axis=1))
+
+
+def row_norm_rows(W, A, B, s, rows) -> np.ndarray:
+    """``row_norm`` restricted to the output channels listed in ``rows``.
+
+    Same definition, evaluated only for a sample of rows so that full-size
+    problems can be checked one row at a time.
+    """
+    rows = np.asarray(rows, dtype=np.int64)
+    W_rows = _f64(W)[rows]
+    B_rows = _f64(B)[rows]
+    return row_norm(W_rows, A, B_rows, s)
+
+
+def magnitude_scale(m, n) -> np.ndarray:
+    """``g = m / n`` (fp64, IEEE semantics for ``n == 0``).
+
+    DoRA summary page, Method: the direction is normalised and rescaled by the
+    learned magnitude.
+    """
+    with np.errstate(divide="ignore", invalid="ignore"):
+        return _f64(m) / _f64(n)
+
+
+def compose_forward(base, lora, m, n, s) -> np.ndarray:
+    """``y = g * (base + s * lora)`` broadcast over tokens.
+
+    Scaling DoRA, Abstract: the DoRA composition of the base output, the LoRA
+    output and the magnitude rescaling.  ``base = x W^T`` and
+    ``lora = x A^T B^T`` (unscaled) are ``[tokens, d_out]``.
+    """
+    base, lora = _f64(base), _f64(lora)
+    g = magnitude_scale(m, n)
+    return g[None, :] * (base + float(s) * lora)
+
+
+def compose_backward(dy, base, lora, m, n, s):
+    """Gradients of ``y = (m / n) * (base + s * lora)`` with ``n`` constant.
+
+    Returns ``(d_base, d_lora, d_m)``:
+      d_base = g * dy,  d_lora = s * g * dy,
+      d_m_i  = sum_t dy[t, i] * (base[t, i] + s * lora[t, i]) / n_i.
+    Chain rule on the forward definition above (Scaling DoRA, Abstract,
+    "gradient computation"), with the norm detached.
+    """
+    dy, base, lora = _f64(dy), _f64(base), _f64(lora)
+    s = float(s)
+    g = magnitude_scale(m, n)
+    d_base = g[None, :] * dy
+    d_lora = s * g[None, :] * dy
+    with np.errstate(divide="ignore", invalid="ignore"):
+        d_m = np.sum(dy * (base + s * lora), axis=0) / _f64(n)
+    return d_base, d_lora, d_m
+
+
+def compose_backward_columns(dy, base, lora, m, n, s, cols) -> np.ndarray:
+    """``d_m`` of ``compose_backward`` for the output channels in ``cols``.
+
+    ``dy``/``base``/``lora`` are the full ``[tokens, d_out]`` arrays (or any
+    array indexable by column); only the listed columns are reduced.
+    """
+    cols = np.asarray(cols, dtype=np.int64)
+    dy_c = _f64(np.asarray(dy)[:, cols])
+    base_c = _f64(np.asarray(base)[:, cols])
+    lora_c = _f64(np.asarray(lora)[:, cols])
+    _, _, d_m = compose_backward(dy_c, base_c, lora_c, _f64(m)[cols], _f64(n)[cols], s)
+    return d_m
