@@ -1,0 +1,455 @@
+#!/usr/bin/env python
+"""Benchmark of the DoRA hot path on B200: factored row norm + fused compose
+forward + compose backward on the 8192 x 8192, r = 384, bf16 module with
+8192 tokens (synthetic, seeded inputs).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...        (N > 1)
+
+One step = dora_factored_norm -> dora_compose_fwd -> dora_compose_bwd on
+inputs already resident in HBM.  The headline value is the factored norm's
+TFLOP/s (algorithmic FLOPs over the norm launches' CUDA-event time, summed
+over ranks); compose forward / backward HBM GB/s and every kernel's
+roofline fraction ride along in the same JSON line.  Multi-GPU runs are
+independent replicas (weak scaling): the path has no exchange step.
+
+``--impl reference`` times the fp64 CPU oracle (the reference arm) on the
+host cores on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from factored_weight_norm_b200 import workloads as WL  # noqa: E402
+
+METRIC = "factored-norm TFLOP/s + fused-compose HBM GB/s (d=8192, r=384, bf16), % roofline"
+# bounded oracle sample per step: norm rows, compose tokens (about 1 s of CPU work)
+ORACLE_SAMPLE = (1024, 512)
+ORACLE_REPS = 10
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------ algorithmic work
+def norm_flops(d_out, d_in, r):
+    """Fixed count: cross GEMM + Gram + Gram quadratic form + base norm + row dot."""
+    return 2 * d_out * d_in * r + 2 * r * r * d_in + 2 * d_out * r * r + 2 * d_out * d_in + 2 * d_out * r
+
+
+def norm_bytes(d_out, d_in, r, e=2):
+    return e * (d_out * d_in + r * d_in + d_out * r) + 4 * d_out
+
+
+def fwd_bytes(T, d_out, e=2):
+    return 3 * e * T * d_out + 8 * d_out
+
+
+def bwd_bytes(T, d_out, e=2):
+    return 5 * e * T * d_out + 12 * d_out
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_digest():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "factored_weight_norm_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic():
+    """DRAM bytes per launch from the committed ncu summary, valid only for the
+    kernel sources it was captured from."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    out = {}
+    if not os.path.exists(p):
+        return out
+    digest = source_digest()
+    for line in open(p):
+        parts = line.split()
+        if len(parts) >= 4 and not line.startswith("#") and parts[1] == digest:
+            out[parts[0]] = {"bytes": float(parts[2]), "workload": parts[3]}
+    return out
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        self.path = f"/tmp/dora_clocks_{os.getpid()}.csv"
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                cur, mx, pw = float(f[1]), float(f[2]), float(f[3])
+            except ValueError:
+                continue
+            smax = mx
+            if pw > 250 or cur > 0.5 * mx:  # under load
+                sm.append(cur)
+                for nm, v in zip(names, f[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "samples_under_load": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    from factored_weight_norm_b200 import dora as D
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = WL.WORKLOADS[args.workload]
+    T, d_out, d_in, r, s = wl.tokens, wl.d_out, wl.d_in, wl.r, wl.s
+    W, A, B, m = WL.make_weights(wl, dev)
+    _, base, lora = WL.make_activations(wl, W, A, B, dev)
+    dy = WL.make_grad(wl, dev)
+    n = torch.empty(d_out, dtype=torch.float32, device=dev)
+    y = torch.empty_like(base)
+    d_base = torch.empty_like(base)
+    d_lora = torch.empty_like(base)
+    d_m = torch.empty(d_out, dtype=torch.float32, device=dev)
+    ws_n = torch.empty(D.dora_factored_norm_workspace_size(d_out, d_in, r), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(D.dora_compose_bwd_workspace_size(T, d_out), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        D.dora_factored_norm(W, A, B, s, n_out=n, workspace=ws_n)
+        if ev is not None:
+            ev[1].record(stream)
+        D.dora_compose_fwd(base, lora, m, n, s, y=y)
+        if ev is not None:
+            ev[2].record(stream)
+        D.dora_compose_bwd(dy, base, lora, m, n, s, d_base, d_lora, d_m, ws_b)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if D.dora_device_status() != D.DORA_OK:
+        raise RuntimeError("device status not OK after warm-up")
+
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        step(evs[k])
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop() if sampler else None
+    status = D.dora_device_status()
+
+    t_norm = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps * 1e-3
+    t_fwd = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps * 1e-3
+    t_bwd = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps * 1e-3
+    t_total = evs[0][0].elapsed_time(evs[-1][3]) * 1e-3
+    times = torch.tensor([t_total, t_norm, t_fwd, t_bwd], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
+    t_total, t_norm, t_fwd, t_bwd = times.tolist()
+
+    # ---- end to end through the Python API with pinned host buffers
+    e2e = run_e2e(args, D, dev, wl, W, A, B, m, base, lora, dy, n, y, d_base, d_lora, d_m, ws_n, ws_b, world)
+    return dict(t_total=t_total, t_norm=t_norm, t_fwd=t_fwd, t_bwd=t_bwd, clocks=clocks, status=status, e2e=e2e,
+                wl=wl)
+
+
+def run_e2e(args, D, dev, wl, W, A, B, m, base, lora, dy, n, y, d_base, d_lora, d_m, ws_n, ws_b, world):
+    T, d_out, s = wl.tokens, wl.d_out, wl.s
+    h = {k: v.cpu().pin_memory() for k, v in dict(W=W, A=A, B=B, m=m, base=base, lora=lora, dy=dy).items()}
+    o = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in
+         dict(n=n, y=y, d_base=d_base, d_lora=d_lora, d_m=d_m).items()}
+    h2d = sum(v.numel() * v.element_size() for v in h.values())
+    d2h = sum(v.numel() * v.element_size() for v in o.values())
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        rec = (lambda i: ev[i].record(stream)) if ev is not None else (lambda i: None)
+        rec(0)
+        W.copy_(h["W"], non_blocking=True)
+        A.copy_(h["A"], non_blocking=True)
+        B.copy_(h["B"], non_blocking=True)
+        D.dora_factored_norm(W, A, B, s, n_out=n, workspace=ws_n)
+        o["n"].copy_(n, non_blocking=True)
+        rec(1)
+        m.copy_(h["m"], non_blocking=True)
+        base.copy_(h["base"], non_blocking=True)
+        lora.copy_(h["lora"], non_blocking=True)
+        D.dora_compose_fwd(base, lora, m, n, s, y=y)
+        o["y"].copy_(y, non_blocking=True)
+        rec(2)
+        dy.copy_(h["dy"], non_blocking=True)
+        D.dora_compose_bwd(dy, base, lora, m, n, s, d_base, d_lora, d_m, ws_b)
+        o["d_base"].copy_(d_base, non_blocking=True)
+        o["d_lora"].copy_(d_lora, non_blocking=True)
+        o["d_m"].copy_(d_m, non_blocking=True)
+        rec(3)
+
+    for _ in range(max(1, min(args.warmup, 2))):
+        step()
+    torch.cuda.synchronize()
+    k = max(1, min(args.steps, 5))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(k)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    for i in range(k):
+        step(evs[i])
+    torch.cuda.synchronize()
+    t = torch.tensor([sum(e[0].elapsed_time(e[1]) for e in evs) / k * 1e-3,
+                      sum(e[1].elapsed_time(e[2]) for e in evs) / k * 1e-3,
+                      sum(e[2].elapsed_time(e[3]) for e in evs) / k * 1e-3], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    t_norm, t_fwd, t_bwd = t.tolist()
+    return dict(t_norm=t_norm, t_fwd=t_fwd, t_bwd=t_bwd, h2d=h2d, d2h=d2h, steps=k)
+
+
+# ------------------------------------------------------- oracle (CPU) arm
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        return max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def time_oracle(wl, norm_rows, compose_tokens, seed=0):
+    """Oracle norm on `norm_rows` rows and compose fwd/bwd on `compose_tokens`
+    tokens of the workload; returns (norm TFLOP/s, fwd GB/s, bwd GB/s, sample)."""
+    import numpy as np
+
+    import oracle
+
+    W, A, B, m = WL.make_weights(wl.with_(d_out=norm_rows))
+    W64, A64, B64 = (t.double().numpy() for t in (W, A, B))
+    t0 = time.perf_counter()
+    n = oracle.row_norm(W64, A64, B64, wl.s)
+    t_norm = time.perf_counter() - t0
+    rng = np.random.default_rng(seed)
+    T, d = compose_tokens, wl.d_out
+    base = rng.standard_normal((T, d)).astype(np.float32).astype(np.float64)
+    lora = rng.standard_normal((T, d)).astype(np.float32).astype(np.float64) * 0.02
+    dy = rng.standard_normal((T, d)).astype(np.float32).astype(np.float64)
+    mm = np.ones(d)
+    nn = np.ones(d) * (1 + 1e-4)
+    t0 = time.perf_counter()
+    oracle.compose_forward(base, lora, mm, nn, wl.s)
+    t_fwd = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.compose_backward(dy, base, lora, mm, nn, wl.s)
+    t_bwd = time.perf_counter() - t0
+    del n
+    tf = norm_flops(norm_rows, wl.d_in, wl.r) / t_norm / 1e12
+    return dict(
+        norm_tflops=tf, fwd_gbs=fwd_bytes(T, d) / t_fwd / 1e9, bwd_gbs=bwd_bytes(T, d) / t_bwd / 1e9,
+        t=t_norm + t_fwd + t_bwd,
+        sample=f"norm on {norm_rows} of {wl.d_out} rows (full d_in, r); compose fwd/bwd on {T} of {wl.tokens} tokens",
+    )
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    wl = WL.WORKLOADS[args.workload]
+    for _ in range(args.warmup):
+        time_oracle(wl, *ORACLE_SAMPLE)
+    res = []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        res.append(time_oracle(wl, *ORACLE_SAMPLE))
+    wall = time.perf_counter() - t0
+    v = statistics.median(r["norm_tflops"] for r in res)
+    cores = oracle_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": wall / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "d_out": wl.d_out, "d_in": wl.d_in, "r": wl.r, "tokens": wl.tokens,
+                   "s": wl.s, "sample": res[0]["sample"]},
+        "compose": {"fwd_gbs": statistics.median(r["fwd_gbs"] for r in res),
+                    "bwd_gbs": statistics.median(r["bwd_gbs"] for r in res)},
+        "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": res[0]["sample"]},
+        "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WL.HEADLINE.name, choices=sorted(WL.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed CPU oracle sample")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    if world > 1:
+        import datetime
+
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    res = run_ours(args, rank, world, local_rank)
+    wl = res["wl"]
+    N = world
+    F = norm_flops(wl.d_out, wl.d_in, wl.r)
+    Bn = norm_bytes(wl.d_out, wl.d_in, wl.r)
+    Bf = fwd_bytes(wl.tokens, wl.d_out)
+    Bb = bwd_bytes(wl.tokens, wl.d_out)
+    peaks, peak_src = load_peaks()
+    traffic = load_traffic()
+
+    def roof(kernel, t, work, bound):
+        if bound == "tensor":
+            ach = work / t / 1e12
+            pk = peaks["bf16_tflops"]
+            unit = "TFLOP/s"
+        else:
+            ach = work / t / 1e9
+            pk = peaks["hbm_gbs"]
+            unit = "GB/s"
+        tr = traffic.get(kernel)
+        return {"kernel": kernel, "bound": bound, "achieved": ach, "peak": pk, "unit": unit, "frac": ach / pk,
+                "traffic": tr["bytes"] if tr else None, "peak_source": f"{peak_src} (burst)" if bound == "tensor" else peak_src,
+                "time_us": t * 1e6}
+
+    # norm bound: slower of FLOPs at tensor peak and bytes at HBM bandwidth
+    norm_bound = "tensor" if F / (peaks["bf16_tflops"] * 1e12) >= Bn / (peaks["hbm_gbs"] * 1e9) else "hbm"
+    rl = [
+        roof("norm", res["t_norm"], F if norm_bound == "tensor" else Bn, norm_bound),
+        roof("compose_fwd", res["t_fwd"], Bf, "hbm"),
+        roof("compose_bwd", res["t_bwd"], Bb, "hbm"),
+    ]
+    dominant = max(rl, key=lambda x: x["time_us"])
+    e2e = res["e2e"]
+    e2e_norm = F * N / (e2e["t_norm"]) / 1e12
+
+    cpu = None
+    if rank == 0 and N == 1 and not args.no_cpu_baseline:
+        obs = [time_oracle(wl, *ORACLE_SAMPLE) for _ in range(ORACLE_REPS)]
+        cpu = {"value": statistics.median(o["norm_tflops"] for o in obs), "unit": "TFLOP/s",
+               "cores": oracle_threads(), "kind": "oracle",
+               "sample": f"{obs[0]['sample']}; median of {ORACLE_REPS} repetitions",
+               "cpu_seconds": sum(o["t"] for o in obs),
+               "compose_fwd_gbs": statistics.median(o["fwd_gbs"] for o in obs),
+               "compose_bwd_gbs": statistics.median(o["bwd_gbs"] for o in obs)}
+
+    launches_per_step = 3 + 1 + 1  # gram, gram_reduce, norm; compose fwd; compose bwd
+    if rank == 0:
+        line = {
+            "metric": METRIC,
+            "value": F * N / res["t_norm"] / 1e12,
+            "unit": "TFLOP/s",
+            "n_gpus": N,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": res["t_total"] / args.steps * 1e3,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "d_out": wl.d_out, "d_in": wl.d_in, "r": wl.r, "tokens": wl.tokens,
+                       "s": wl.s, "parallelism": f"replicas x{N}",
+                       "l2": "no flush: each step streams > 1 GB (W 134 MB, 3 activation reads + 3 writes of 134 MB)"},
+            "value_basis": "norm FLOPs x ranks / max-over-ranks mean CUDA-event time of the norm launches in the timed steps",
+            "compose": {
+                "fwd": {"value": Bf * N / res["t_fwd"] / 1e9, "unit": "GB/s", "frac": rl[1]["frac"],
+                        "time_us": res["t_fwd"] * 1e6},
+                "bwd": {"value": Bb * N / res["t_bwd"] / 1e9, "unit": "GB/s", "frac": rl[2]["frac"],
+                        "time_us": res["t_bwd"] * 1e6},
+            },
+            "norm": {"tflops": F / res["t_norm"] / 1e12, "frac": rl[0]["frac"], "bound": norm_bound,
+                     "time_us": res["t_norm"] * 1e6, "flops": F, "bytes": Bn},
+            "roofline": {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
+                        | {"kernel": dominant["kernel"], "peak_source": dominant["peak_source"]},
+            "rooflines": rl,
+            "step_roofline_frac": (
+                max(F / (peaks["bf16_tflops"] * 1e12), Bn / (peaks["hbm_gbs"] * 1e9))
+                + Bf / (peaks["hbm_gbs"] * 1e9) + Bb / (peaks["hbm_gbs"] * 1e9)) / (res["t_total"] / args.steps),
+            "e2e": {"value": e2e_norm, "unit": "TFLOP/s", "h2d_bytes_per_step": e2e["h2d"],
+                    "d2h_bytes_per_step": e2e["d2h"], "steps": e2e["steps"],
+                    "basis": "norm FLOPs / (H2D of W, A, B + norm + D2H of n), pinned host buffers",
+                    "compose_fwd_gbs": Bf * N / e2e["t_fwd"] / 1e9, "compose_bwd_gbs": Bb * N / e2e["t_bwd"] / 1e9},
+            "cpu_baseline": cpu,
+            "gpu_launches": launches_per_step * args.steps,
+            "memset_nodes": args.steps,
+            "clocks": res["clocks"],
+            "device_status": res["status"],
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

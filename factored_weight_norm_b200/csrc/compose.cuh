@@ -1,0 +1,235 @@
+// compose.cuh - fused DoRA compose forward / backward (memory-bound).
+//
+// "Scaling DoRA: High-Rank Adaptation via Factored Norms and Fused Kernels",
+// Abstract: the DoRA composition runs as one pass over the activations, in a
+// form that stays accurate when the magnitude rescaling g = m / n is close to 1.
+//
+// Forward, per output channel i (fp32, never rounded to the activation type):
+//   g = m / n,  delta = (m - n) / n   (m - n is exact when m / n is in [1/2, 2])
+//   y = base + (delta * base + g * s * lora)        one final rounding
+// Backward with n constant:
+//   d_base = g * dy,  d_lora = (g * s) * dy,
+//   d_m    = (sum_t dy * (base + s * lora)) / n
+//
+// Both kernels stream 16-byte vectors (8 bf16 or 4 fp32), coalesced along the
+// contiguous d_out axis; each thread keeps its channels' g / delta in
+// registers for all the rows it visits.  The backward carries the token sum
+// in fp32 registers, folds the two half-warps with a shuffle and the eight
+// warps through shared memory, writes one partial per (row chunk, channel),
+// and the last CTA of each column strip adds the chunks in fixed order.
+#pragma once
+
+#include "sm100_ptx.cuh"
+
+namespace dora {
+
+template <typename T, int VEC>
+struct VecIO;
+
+template <>
+struct VecIO<__nv_bfloat16, 8> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[8]) {
+    const uint4 u = ld_stream_u4(p);
+    v[0] = bf16_lo(u.x);
+    v[1] = bf16_hi(u.x);
+    v[2] = bf16_lo(u.y);
+    v[3] = bf16_hi(u.y);
+    v[4] = bf16_lo(u.z);
+    v[5] = bf16_hi(u.z);
+    v[6] = bf16_lo(u.w);
+    v[7] = bf16_hi(u.w);
+  }
+  static __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&v)[8]) {
+    uint4 u;
+    u.x = pack2(v[0], v[1]);
+    u.y = pack2(v[2], v[3]);
+    u.z = pack2(v[4], v[5]);
+    u.w = pack2(v[6], v[7]);
+    st_stream_u4(p, u);
+  }
+};
+
+template <>
+struct VecIO<float, 4> {
+  static __device__ __forceinline__ void load(const float* p, float (&v)[4]) {
+    const uint4 u = ld_stream_u4(p);
+    v[0] = __uint_as_float(u.x);
+    v[1] = __uint_as_float(u.y);
+    v[2] = __uint_as_float(u.z);
+    v[3] = __uint_as_float(u.w);
+  }
+  static __device__ __forceinline__ void store(float* p, const float (&v)[4]) {
+    st_stream_u4(p, make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]),
+                               __float_as_uint(v[3])));
+  }
+};
+
+template <>
+struct VecIO<float, 1> {
+  static __device__ __forceinline__ void load(const float* p, float (&v)[1]) { v[0] = __ldg(p); }
+  static __device__ __forceinline__ void store(float* p, const float (&v)[1]) { p[0] = v[0]; }
+};
+
+// ------------------------------------------------------------------ forward
+template <typename T, int VEC>
+__global__ void __launch_bounds__(256) compose_fwd_kernel(const T* __restrict__ base, const T* __restrict__ lora,
+                                                          const float* __restrict__ m,
+                                                          const float* __restrict__ n, float s,
+                                                          long long tokens, long long nvec, long long d_out,
+                                                          T* __restrict__ y, long long rows_per_cta) {
+  const long long v = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+  if (v >= nvec) return;
+  const long long col = v * VEC;
+  float delta[VEC], gs[VEC];
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) {
+    const float mm = __ldg(m + col + e), nn = __ldg(n + col + e);
+    delta[e] = (mm - nn) / nn;
+    gs[e] = (mm / nn) * s;
+  }
+  const long long row0 = blockIdx.y * rows_per_cta;
+  const long long row1 = min(tokens, row0 + rows_per_cta);
+  long long row = row0;
+  constexpr int U = 4;
+  for (; row + U <= row1; row += U) {
+    float b[U][VEC], l[U][VEC];
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      VecIO<T, VEC>::load(base + (row + k) * d_out + col, b[k]);
+      VecIO<T, VEC>::load(lora + (row + k) * d_out + col, l[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      float o[VEC];
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) o[e] = b[k][e] + fmaf(delta[e], b[k][e], gs[e] * l[k][e]);
+      VecIO<T, VEC>::store(y + (row + k) * d_out + col, o);
+    }
+  }
+  for (; row < row1; ++row) {
+    float b[VEC], l[VEC], o[VEC];
+    VecIO<T, VEC>::load(base + row * d_out + col, b);
+    VecIO<T, VEC>::load(lora + row * d_out + col, l);
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) o[e] = b[e] + fmaf(delta[e], b[e], gs[e] * l[e]);
+    VecIO<T, VEC>::store(y + row * d_out + col, o);
+  }
+}
+
+// ----------------------------------------------------------------- backward
+constexpr int kBwdThreads = 256;  // 8 warps; a half-warp spans 16 vectors of one row
+constexpr int kBwdVecs = 16;      // vectors (column groups) per CTA strip
+constexpr int kBwdSlots = 16;     // rows visited concurrently by one CTA
+
+template <typename T, int VEC>
+__global__ void __launch_bounds__(kBwdThreads) compose_bwd_kernel(
+    const T* __restrict__ dy, const T* __restrict__ base, const T* __restrict__ lora, const float* __restrict__ m,
+    const float* __restrict__ n, float s, long long tokens, long long nvec, long long d_out, T* __restrict__ d_base,
+    T* __restrict__ d_lora, float* __restrict__ partial, int* __restrict__ counters, float* __restrict__ d_m,
+    long long rows_per_chunk) {
+  __shared__ float red[kBwdThreads / 32][kBwdVecs][VEC];
+  __shared__ int is_last;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int half = lane >> 4, vi = lane & 15;
+  const int slot = warp * 2 + half;
+  const long long v = blockIdx.x * static_cast<long long>(kBwdVecs) + vi;
+  const bool valid = v < nvec;
+  const long long col = v * VEC;
+
+  float g[VEC], gs[VEC], acc[VEC];
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) {
+    acc[e] = 0.f;
+    g[e] = 0.f;
+    gs[e] = 0.f;
+  }
+  if (valid) {
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+      g[e] = __ldg(m + col + e) / __ldg(n + col + e);
+      gs[e] = g[e] * s;
+    }
+    const long long row0 = blockIdx.y * rows_per_chunk;
+    const long long row1 = min(tokens, row0 + rows_per_chunk);
+    long long row = row0 + slot;
+    for (; row + kBwdSlots < row1; row += 2 * kBwdSlots) {
+      float a0[VEC], b0[VEC], l0[VEC], a1[VEC], b1[VEC], l1[VEC];
+      const long long o0 = row * d_out + col, o1 = (row + kBwdSlots) * d_out + col;
+      VecIO<T, VEC>::load(dy + o0, a0);
+      VecIO<T, VEC>::load(base + o0, b0);
+      VecIO<T, VEC>::load(lora + o0, l0);
+      VecIO<T, VEC>::load(dy + o1, a1);
+      VecIO<T, VEC>::load(base + o1, b1);
+      VecIO<T, VEC>::load(lora + o1, l1);
+      float db[VEC], dl[VEC];
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        db[e] = g[e] * a0[e];
+        dl[e] = gs[e] * a0[e];
+        acc[e] = fmaf(a0[e], fmaf(s, l0[e], b0[e]), acc[e]);
+      }
+      VecIO<T, VEC>::store(d_base + o0, db);
+      VecIO<T, VEC>::store(d_lora + o0, dl);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        db[e] = g[e] * a1[e];
+        dl[e] = gs[e] * a1[e];
+        acc[e] = fmaf(a1[e], fmaf(s, l1[e], b1[e]), acc[e]);
+      }
+      VecIO<T, VEC>::store(d_base + o1, db);
+      VecIO<T, VEC>::store(d_lora + o1, dl);
+    }
+    for (; row < row1; row += kBwdSlots) {
+      float a0[VEC], b0[VEC], l0[VEC], db[VEC], dl[VEC];
+      const long long o0 = row * d_out + col;
+      VecIO<T, VEC>::load(dy + o0, a0);
+      VecIO<T, VEC>::load(base + o0, b0);
+      VecIO<T, VEC>::load(lora + o0, l0);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        db[e] = g[e] * a0[e];
+        dl[e] = gs[e] * a0[e];
+        acc[e] = fmaf(a0[e], fmaf(s, l0[e], b0[e]), acc[e]);
+      }
+      VecIO<T, VEC>::store(d_base + o0, db);
+      VecIO<T, VEC>::store(d_lora + o0, dl);
+    }
+  }
+
+  // fold the two half-warps (same columns, different rows), then the 8 warps
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
+  if (half == 0) {
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) red[warp][vi][e] = acc[e];
+  }
+  __syncthreads();
+  const int t = threadIdx.x;
+  const long long tcol = blockIdx.x * static_cast<long long>(kBwdVecs) * VEC + t;
+  const bool t_ok = t < kBwdVecs * VEC && tcol < d_out;
+  if (t_ok) {
+    float sum = 0.f;
+#pragma unroll
+    for (int w = 0; w < kBwdThreads / 32; ++w) sum += red[w][t / VEC][t % VEC];
+    partial[blockIdx.y * d_out + tcol] = sum;
+  }
+  __threadfence();
+  __syncthreads();
+  if (t == 0) is_last = (atomicAdd(&counters[blockIdx.x], 1) == static_cast<int>(gridDim.y) - 1);
+  __syncthreads();
+  if (is_last) {
+    __threadfence();
+    if (t_ok) {
+      float total = 0.f;
+      for (unsigned c = 0; c < gridDim.y; ++c) total += ld_cg_f32(&partial[c * d_out + tcol]);
+      d_m[tcol] = total / __ldg(n + tcol);
+    }
+    if (t == 0) counters[blockIdx.x] = 0;
+  }
+}
+
+}  // namespace dora

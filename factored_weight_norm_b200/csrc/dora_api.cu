@@ -1,0 +1,410 @@
+// dora_api.cu - the C ABI declared in include/dora.h: argument validation,
+// launch planning, TMA descriptor encoding and kernel launches.
+//
+// The library never allocates device memory: every buffer, including the
+// workspace, comes from the caller.  All work is enqueued on the caller's
+// stream.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/dora.h"
+#include "compose.cuh"
+#include "norm_simt.cuh"
+#include "norm_tc.cuh"
+
+namespace dora {
+
+// Device-side status word: kernels write DORA_ERR_TIMEOUT here when a bounded
+// wait gives up.  One per device (a __device__ variable lives in every
+// context that loads the library).
+__device__ int g_status = 0;
+
+namespace {
+
+constexpr long long kWaitLimitCycles = 2000000000LL;  // ~1 s at B200 clocks
+constexpr int kMaxGrid = 1024;                         // bound on the persistent grid
+constexpr int kMaxGramSplits = 32;
+constexpr int kMaxBwdChunks = 64;
+constexpr int kCtasPerSm = 8;  // 256-thread CTAs that fill an SM's 2048 thread slots
+constexpr int kMaxDevices = 64;
+constexpr int64_t kMaxRank = 4096;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
+
+struct DeviceInfo {
+  bool ready = false;
+  int num_sms = 0;
+  int smem_optin = 0;
+  int* status = nullptr;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+// Per-device set-up, done once with that device current.
+int device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DORA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return DORA_ERR_CUDA;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return DORA_ERR_CUDA;
+    d.status = static_cast<int*>(p);
+    if (cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+      return DORA_ERR_CUDA;
+    if (cudaFuncSetAttribute(norm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin) != cudaSuccess)
+      return DORA_ERR_CUDA;
+    if (cudaFuncSetAttribute(gram_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin) != cudaSuccess)
+      return DORA_ERR_CUDA;
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return DORA_ERR_CUDA;
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    d.ready = true;
+  }
+  *out = &d;
+  return DORA_OK;
+}
+
+// 2-D bf16 tensor map over a row-major [rows, cols] matrix, 64 x 128 boxes,
+// 128-byte swizzle, zero fill outside the matrix.
+int make_map(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols) {
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(kBoxRows)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DORA_OK : DORA_ERR_CUDA;
+}
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// ------------------------------------------------------------ norm planning
+struct TcPlan {
+  int m_tiles, n_chunks, chunk_n, kb_main, kb_ext, kb_total;
+  long long units;
+  int gram_tiles, gram_splits_max;
+  size_t off_gs, off_gp, off_part, off_cnt, total;
+};
+
+TcPlan plan_tc(int64_t d_out, int64_t d_in, int64_t r) {
+  TcPlan p{};
+  p.m_tiles = static_cast<int>(cdiv(d_out, kBM));
+  p.n_chunks = static_cast<int>(cdiv(r, kMaxChunkN));
+  p.chunk_n = static_cast<int>(align_up(static_cast<size_t>(cdiv(r, p.n_chunks)), 16));
+  p.kb_main = static_cast<int>(cdiv(d_in, kBK));
+  p.kb_ext = static_cast<int>(cdiv(r, kBK));
+  p.kb_total = p.kb_main + p.kb_ext;
+  p.units = static_cast<long long>(p.m_tiles) * p.n_chunks * p.kb_total;
+  const int nt = static_cast<int>(cdiv(r, kBoxRows));
+  p.gram_tiles = nt * (nt + 1) / 2;
+  p.gram_splits_max = std::max(1, std::min({kMaxGramSplits, 160 / p.gram_tiles, p.kb_main}));
+  size_t off = 0;
+  p.off_gs = off;
+  off = align_up(off + static_cast<size_t>(r) * r * 2, 1024);
+  p.off_gp = off;
+  off = align_up(off + static_cast<size_t>(p.gram_splits_max) * p.gram_tiles * kBoxRows * kBoxRows * 4, 256);
+  p.off_part = off;
+  off = align_up(off + static_cast<size_t>(kMaxGrid + p.m_tiles * p.n_chunks) * kBM * 4, 256);
+  p.off_cnt = off;
+  off = align_up(off + static_cast<size_t>(p.m_tiles) * 4, 256);
+  p.total = off;
+  return p;
+}
+
+size_t f32_norm_ws(int64_t r) { return align_up(static_cast<size_t>(r) * r * 4, 256) + 256; }
+
+int launch_error() { return cudaGetLastError() == cudaSuccess ? DORA_OK : DORA_ERR_CUDA; }
+
+int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_t d_in, int64_t r, float s,
+              float* n_out, void* ws, cudaStream_t st, DeviceInfo* dev) {
+  const TcPlan p = plan_tc(d_out, d_in, r);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  __nv_bfloat16* Gs = reinterpret_cast<__nv_bfloat16*>(w + p.off_gs);
+  float* Gp = reinterpret_cast<float*>(w + p.off_gp);
+  float* part = reinterpret_cast<float*>(w + p.off_part);
+  int* cnt = reinterpret_cast<int*>(w + p.off_cnt);
+
+  CUtensorMap tmW, tmA, tmB, tmG;
+  if (make_map(&tmW, W, d_out, d_in) || make_map(&tmA, A, r, d_in) || make_map(&tmB, B, d_out, r) ||
+      make_map(&tmG, Gs, r, r))
+    return DORA_ERR_CUDA;
+
+  // 1) Gram partial tiles, 2) reduce to bf16 (s/2) G and zero the counters
+  GramArgs ga{};
+  ga.r = static_cast<int>(r);
+  ga.kb_main = p.kb_main;
+  ga.splits = std::max(1, std::min(p.gram_splits_max, dev->num_sms / p.gram_tiles));
+  ga.n_tiles = static_cast<int>(cdiv(r, kBoxRows));
+  ga.wait_limit = kWaitLimitCycles;
+  ga.partial = Gp;
+  ga.status = dev->status;
+  const size_t gram_smem = kGramStages * kGramStageBytes + (2 * kGramStages + 1) * 8 + 16 + 1024;
+  gram_tc_kernel<<<p.gram_tiles * ga.splits, kNormThreads, gram_smem, st>>>(tmA, ga);
+  if (launch_error()) return DORA_ERR_CUDA;
+  const long long rr = static_cast<long long>(r) * r;
+  const int red_blocks = static_cast<int>(std::max<long long>(cdiv(p.m_tiles, 256), std::min<long long>(cdiv(rr, 256), 4 * dev->num_sms)));
+  gram_reduce_kernel<<<red_blocks, 256, 0, st>>>(Gp, ga.splits, static_cast<int>(r), 0.5f * s, Gs, cnt, p.m_tiles);
+  if (launch_error()) return DORA_ERR_CUDA;
+
+  // 3) persistent stream-K GEMM with the fused norm epilogue
+  NormArgs na{};
+  na.d_out = static_cast<int>(d_out);
+  na.d_in = static_cast<int>(d_in);
+  na.r = static_cast<int>(r);
+  na.m_tiles = p.m_tiles;
+  na.n_chunks = p.n_chunks;
+  na.chunk_n = p.chunk_n;
+  na.kb_main = p.kb_main;
+  na.kb_total = p.kb_total;
+  na.units = p.units;
+  na.n_tile_bytes = static_cast<uint32_t>(cdiv(p.chunk_n, kBoxRows) * kBoxBytes);
+  na.stage_bytes = kBoxBytes + na.n_tile_bytes;
+  const size_t fixed = 1024 + 64 + 16;
+  na.stages = static_cast<int>(std::min<size_t>(kMaxStages, (dev->smem_optin - fixed) / (na.stage_bytes + 16)));
+  if (na.stages < 2) return DORA_ERR_UNSUPPORTED;
+  uint32_t cols = 32;
+  while (cols < static_cast<uint32_t>(p.chunk_n)) cols <<= 1;
+  na.tmem_cols = cols;
+  na.two_s = 2.0f * s;
+  na.wait_limit = kWaitLimitCycles;
+  na.B = static_cast<const __nv_bfloat16*>(B);
+  na.partials = part;
+  na.counters = cnt;
+  na.n_out = n_out;
+  na.status = dev->status;
+  const int grid = static_cast<int>(std::min<long long>({static_cast<long long>(dev->num_sms), p.units, kMaxGrid}));
+  const size_t smem = static_cast<size_t>(na.stages) * na.stage_bytes + (2 * na.stages + 3) * 8 + 16 + 1024;
+  norm_tc_kernel<<<grid, kNormThreads, smem, st>>>(tmW, tmA, tmB, tmG, na);
+  return launch_error();
+}
+
+}  // namespace
+}  // namespace dora
+
+using namespace dora;
+
+extern "C" {
+
+const char* dora_status_string(int status) {
+  switch (status) {
+    case DORA_OK: return "DORA_OK";
+    case DORA_ERR_INVALID_ARG: return "DORA_ERR_INVALID_ARG: invalid argument";
+    case DORA_ERR_UNSUPPORTED: return "DORA_ERR_UNSUPPORTED: shape, alignment or dtype not supported";
+    case DORA_ERR_WORKSPACE: return "DORA_ERR_WORKSPACE: workspace missing or too small";
+    case DORA_ERR_CUDA: return "DORA_ERR_CUDA: a CUDA runtime call failed";
+    case DORA_ERR_TIMEOUT: return "DORA_ERR_TIMEOUT: a bounded device-side wait gave up";
+    default: return "unknown dora status";
+  }
+}
+
+size_t dora_factored_norm_workspace_size(int64_t d_out, int64_t d_in, int64_t r, dora_dtype dt) {
+  if (d_out < 0 || d_in < 0 || r < 0) return 0;
+  if (dt == DORA_F32) return f32_norm_ws(r);
+  if (dt != DORA_BF16) return 0;
+  if (d_out == 0 || d_in == 0 || r == 0) return 256;
+  return plan_tc(d_out, d_in, r).total;
+}
+
+int dora_factored_norm(const void* W, const void* A, const void* B, int64_t d_out, int64_t d_in, int64_t r, float s,
+                       dora_dtype dt, float* n_out, void* workspace, size_t workspace_bytes, void* stream) {
+  if (dt != DORA_BF16 && dt != DORA_F32) return DORA_ERR_UNSUPPORTED;
+  if (d_out < 0 || d_in < 0 || r < 0) return DORA_ERR_INVALID_ARG;
+  if (d_out > INT32_MAX / 2 || d_in > INT32_MAX / 2 || r > kMaxRank) return DORA_ERR_UNSUPPORTED;
+  if (d_out == 0) return DORA_OK;
+  if (!n_out || (d_in > 0 && !W) || (r > 0 && d_in > 0 && (!A || !B))) return DORA_ERR_INVALID_ARG;
+  if (!aligned(n_out, 4)) return DORA_ERR_UNSUPPORTED;
+  const size_t need = dora_factored_norm_workspace_size(d_out, d_in, r, dt);
+  const bool trivial = (d_in == 0);
+  if (!trivial && (!workspace || workspace_bytes < need)) return DORA_ERR_WORKSPACE;
+  if (!trivial && !aligned(workspace, 256)) return DORA_ERR_UNSUPPORTED;
+  if (dt == DORA_BF16) {
+    if (!trivial && (d_in % 8 != 0 || r % 16 != 0)) return DORA_ERR_UNSUPPORTED;
+    if (!aligned(W, 16) || !aligned(A, 16) || !aligned(B, 16)) return DORA_ERR_UNSUPPORTED;
+  } else {
+    if (!aligned(W, 4) || !aligned(A, 4) || !aligned(B, 4)) return DORA_ERR_UNSUPPORTED;
+  }
+  DeviceInfo* dev = nullptr;
+  if (device_info(&dev)) return DORA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (trivial) {
+    return cudaMemsetAsync(n_out, 0, static_cast<size_t>(d_out) * 4, st) == cudaSuccess ? DORA_OK : DORA_ERR_CUDA;
+  }
+  if (r == 0) {
+    const int blocks = static_cast<int>(cdiv(d_out, 8));
+    if (dt == DORA_BF16)
+      rownorm_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(W), static_cast<int>(d_out),
+                                                            static_cast<int>(d_in), n_out);
+    else
+      rownorm_kernel<float><<<blocks, 256, 0, st>>>(static_cast<const float*>(W), static_cast<int>(d_out),
+                                                    static_cast<int>(d_in), n_out);
+    return launch_error();
+  }
+  if (dt == DORA_BF16) return norm_bf16(W, A, B, d_out, d_in, r, s, n_out, workspace, st, dev);
+  float* G = static_cast<float*>(workspace);
+  const long long pairs = r * (r + 1) / 2;
+  const int gblocks = static_cast<int>(std::min<long long>(cdiv(pairs, 8), 8LL * dev->num_sms));
+  gram_f32_kernel<<<gblocks, 256, 0, st>>>(static_cast<const float*>(A), static_cast<int>(r), static_cast<int>(d_in), G);
+  if (launch_error()) return DORA_ERR_CUDA;
+  norm_f32_kernel<<<static_cast<unsigned>(d_out), 256, 0, st>>>(
+      static_cast<const float*>(W), static_cast<const float*>(A), static_cast<const float*>(B), G,
+      static_cast<int>(d_out), static_cast<int>(d_in), static_cast<int>(r), s, n_out);
+  return launch_error();
+}
+
+int dora_compose_fwd(const void* base_out, const void* lora_out, const float* m, const float* n, float s,
+                     int64_t tokens, int64_t d_out, dora_dtype dt, void* y, void* stream) {
+  if (dt != DORA_BF16 && dt != DORA_F32) return DORA_ERR_UNSUPPORTED;
+  if (tokens < 0 || d_out < 0) return DORA_ERR_INVALID_ARG;
+  if (tokens == 0 || d_out == 0) return DORA_OK;
+  if (!base_out || !lora_out || !m || !n || !y) return DORA_ERR_INVALID_ARG;
+  const int vec_bf16 = 8;
+  int vec = 1;
+  if (dt == DORA_BF16) {
+    if (d_out % vec_bf16 != 0) return DORA_ERR_UNSUPPORTED;
+    if (!aligned(base_out, 16) || !aligned(lora_out, 16) || !aligned(y, 16)) return DORA_ERR_UNSUPPORTED;
+    vec = vec_bf16;
+  } else {
+    if (!aligned(base_out, 4) || !aligned(lora_out, 4) || !aligned(y, 4)) return DORA_ERR_UNSUPPORTED;
+    vec = (d_out % 4 == 0 && aligned(base_out, 16) && aligned(lora_out, 16) && aligned(y, 16)) ? 4 : 1;
+  }
+  if (!aligned(m, 4) || !aligned(n, 4)) return DORA_ERR_UNSUPPORTED;
+  DeviceInfo* dev = nullptr;
+  if (device_info(&dev)) return DORA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long nvec = d_out / vec;
+  const int threads = static_cast<int>(std::min<long long>(256, align_up(static_cast<size_t>(nvec), 32)));
+  const long long gx = cdiv(nvec, threads);
+  if (gx > INT32_MAX) return DORA_ERR_UNSUPPORTED;
+  const long long gy = std::max<long long>(1, std::min<long long>({static_cast<long long>(dev->num_sms) * kCtasPerSm / gx, tokens, 65535}));
+  const long long rows = cdiv(tokens, gy);
+  const long long gy2 = cdiv(tokens, rows);
+  dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy2));
+  if (dt == DORA_BF16)
+    compose_fwd_kernel<__nv_bfloat16, 8><<<grid, threads, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(base_out), static_cast<const __nv_bfloat16*>(lora_out), m, n, s, tokens,
+        nvec, d_out, static_cast<__nv_bfloat16*>(y), rows);
+  else if (vec == 4)
+    compose_fwd_kernel<float, 4><<<grid, threads, 0, st>>>(static_cast<const float*>(base_out),
+                                                           static_cast<const float*>(lora_out), m, n, s, tokens,
+                                                           nvec, d_out, static_cast<float*>(y), rows);
+  else
+    compose_fwd_kernel<float, 1><<<grid, threads, 0, st>>>(static_cast<const float*>(base_out),
+                                                           static_cast<const float*>(lora_out), m, n, s, tokens,
+                                                           nvec, d_out, static_cast<float*>(y), rows);
+  return launch_error();
+}
+
+size_t dora_compose_bwd_workspace_size(int64_t tokens, int64_t d_out) {
+  if (tokens < 0 || d_out < 0) return 0;
+  const size_t strips = static_cast<size_t>(cdiv(std::max<int64_t>(d_out, 1), dora::kBwdVecs));
+  return align_up(strips * 4, 256) + align_up(static_cast<size_t>(kMaxBwdChunks) * std::max<int64_t>(d_out, 1) * 4, 256);
+}
+
+int dora_compose_bwd(const void* dy, const void* base_out, const void* lora_out, const float* m, const float* n,
+                     float s, int64_t tokens, int64_t d_out, dora_dtype dt, void* d_base, void* d_lora, float* d_m,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  if (dt != DORA_BF16 && dt != DORA_F32) return DORA_ERR_UNSUPPORTED;
+  if (tokens < 0 || d_out < 0) return DORA_ERR_INVALID_ARG;
+  if (d_out == 0) return DORA_OK;
+  if (!m || !n || !d_m) return DORA_ERR_INVALID_ARG;
+  if (tokens > 0 && (!dy || !base_out || !lora_out || !d_base || !d_lora)) return DORA_ERR_INVALID_ARG;
+  int vec = 1;
+  if (dt == DORA_BF16) {
+    if (d_out % 8 != 0) return DORA_ERR_UNSUPPORTED;
+    if (tokens > 0 && (!aligned(dy, 16) || !aligned(base_out, 16) || !aligned(lora_out, 16) ||
+                       !aligned(d_base, 16) || !aligned(d_lora, 16)))
+      return DORA_ERR_UNSUPPORTED;
+    vec = 8;
+  } else {
+    const bool a16 = aligned(dy, 16) && aligned(base_out, 16) && aligned(lora_out, 16) && aligned(d_base, 16) &&
+                     aligned(d_lora, 16);
+    if (!aligned(dy, 4) || !aligned(base_out, 4) || !aligned(lora_out, 4) || !aligned(d_base, 4) ||
+        !aligned(d_lora, 4))
+      return DORA_ERR_UNSUPPORTED;
+    vec = (d_out % 4 == 0 && a16) ? 4 : 1;
+  }
+  if (!aligned(m, 4) || !aligned(n, 4) || !aligned(d_m, 4)) return DORA_ERR_UNSUPPORTED;
+  const size_t need = dora_compose_bwd_workspace_size(tokens, d_out);
+  if (!workspace || workspace_bytes < need) return DORA_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return DORA_ERR_UNSUPPORTED;
+  DeviceInfo* dev = nullptr;
+  if (device_info(&dev)) return DORA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (tokens == 0) return cudaMemsetAsync(d_m, 0, static_cast<size_t>(d_out) * 4, st) == cudaSuccess ? DORA_OK : DORA_ERR_CUDA;
+
+  const long long nvec = d_out / vec;
+  const long long strips = cdiv(nvec, kBwdVecs);
+  if (strips > INT32_MAX) return DORA_ERR_UNSUPPORTED;
+  const long long chunks = std::max<long long>(
+      1, std::min<long long>({static_cast<long long>(dev->num_sms) * kCtasPerSm / strips, kMaxBwdChunks,
+                              cdiv(tokens, kBwdSlots)}));
+  const long long rows = cdiv(tokens, chunks);
+  const long long chunks2 = cdiv(tokens, rows);
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  int* cnt = reinterpret_cast<int*>(w);
+  const size_t strips_all = static_cast<size_t>(cdiv(d_out, kBwdVecs));
+  float* part = reinterpret_cast<float*>(w + align_up(strips_all * 4, 256));
+  if (cudaMemsetAsync(cnt, 0, static_cast<size_t>(strips) * 4, st) != cudaSuccess) return DORA_ERR_CUDA;
+  dim3 grid(static_cast<unsigned>(strips), static_cast<unsigned>(chunks2));
+  if (dt == DORA_BF16)
+    compose_bwd_kernel<__nv_bfloat16, 8><<<grid, kBwdThreads, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(dy), static_cast<const __nv_bfloat16*>(base_out),
+        static_cast<const __nv_bfloat16*>(lora_out), m, n, s, tokens, nvec, d_out,
+        static_cast<__nv_bfloat16*>(d_base), static_cast<__nv_bfloat16*>(d_lora), part, cnt, d_m, rows);
+  else if (vec == 4)
+    compose_bwd_kernel<float, 4><<<grid, kBwdThreads, 0, st>>>(
+        static_cast<const float*>(dy), static_cast<const float*>(base_out), static_cast<const float*>(lora_out), m, n,
+        s, tokens, nvec, d_out, static_cast<float*>(d_base), static_cast<float*>(d_lora), part, cnt, d_m, rows);
+  else
+    compose_bwd_kernel<float, 1><<<grid, kBwdThreads, 0, st>>>(
+        static_cast<const float*>(dy), static_cast<const float*>(base_out), static_cast<const float*>(lora_out), m, n,
+        s, tokens, nvec, d_out, static_cast<float*>(d_base), static_cast<float*>(d_lora), part, cnt, d_m, rows);
+  return launch_error();
+}
+
+int dora_device_status(void* stream) {
+  DeviceInfo* dev = nullptr;
+  if (device_info(&dev)) return DORA_ERR_CUDA;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DORA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return DORA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    cudaMemcpyToSymbol(g_status, &zero, sizeof(int));
+  }
+  return v;
+}
+
+int dora_num_sms(void) {
+  int n = 0;
+  if (cudaGetDeviceCount(&n) != cudaSuccess || n == 0) {
+    cudaGetLastError();
+    return 0;
+  }
+  DeviceInfo* dev = nullptr;
+  if (device_info(&dev)) return 0;
+  return dev->num_sms;
+}
+
+}  // extern "C"

@@ -1,0 +1,518 @@
+// norm_tc.cuh - bf16 factored row norm on tcgen05 tensor cores (sm_100a).
+//
+// "Scaling DoRA: High-Rank Adaptation via Factored Norms and Fused Kernels",
+// Abstract: the squared row norm of W + sBA splits into base, cross and Gram
+// terms that need only O(d_out r + r^2) intermediates:
+//
+//   n_i^2 = ||W_i||^2 + 2s <B_i, U_i> + s^2 B_i G B_i^T,  U = W A^T, G = A A^T.
+//
+// Folding the Gram term into the same contraction: with G' = (s/2) G,
+//   V = [W | B] [A | G']^T = W A^T + (s/2) B G     (K extended by r)
+//   n_i^2 = ||W_i||^2 + 2s <B_i, V_i>.
+// So one tensor-core GEMM (M = d_out, N = r, K = d_in + r) with a row-dot
+// epilogue gives every term; W is streamed from HBM exactly once and the
+// [d_out, r] product V never leaves TMEM.
+//
+// Kernels:
+//   gram_tc_kernel     G = A A^T partial tiles (upper triangle, split over K)
+//   gram_reduce_kernel sums the K splits in fixed order, writes bf16 G'
+//   norm_tc_kernel     persistent stream-K GEMM over (M tile, N chunk, K
+//                      block) units; each CTA owns a contiguous unit range.
+//                      Epilogue: ||W_i||^2 from the shared-memory W stages,
+//                      <B_i, V_i> from TMEM; per-(row, segment) scalar
+//                      partials; the last CTA to finish an M tile sums its
+//                      partials in fixed order and writes n = sqrt(max(., 0)).
+#pragma once
+
+#include "sm100_ptx.cuh"
+
+namespace dora {
+
+constexpr int kBM = 128;              // rows per M tile (TMEM lanes)
+constexpr int kBK = 64;               // bf16 along K per 128-byte swizzled row
+constexpr int kBoxRows = 128;         // rows per TMA box
+constexpr int kBoxBytes = kBoxRows * 128;
+constexpr int kNormThreads = 192;     // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kMaxChunkN = 512;       // TMEM columns
+constexpr int kMaxStages = 8;
+constexpr int kStatusTimeout = 5;     // == DORA_ERR_TIMEOUT
+
+struct NormArgs {
+  int d_out, d_in, r;
+  int m_tiles, n_chunks, chunk_n, kb_main, kb_total;
+  long long units;
+  int stages;
+  uint32_t stage_bytes;   // W-side tile + N-side tiles
+  uint32_t n_tile_bytes;  // bytes reserved for the N-side tiles of a stage
+  uint32_t tmem_cols;
+  float two_s;
+  long long wait_limit;
+  const __nv_bfloat16* B;  // [d_out, r], read by the epilogue
+  float* partials;         // [(gridDim.x + m_tiles * n_chunks) * 128]
+  int* counters;           // [m_tiles], zero on entry, left zero on exit
+  float* n_out;            // [d_out]
+  int* status;
+};
+
+// Owner CTA of unit u when U units are split into G contiguous ranges
+// [floor(c U / G), floor((c + 1) U / G)).
+__host__ __device__ __forceinline__ int stream_k_owner(long long u, long long U, int G) {
+  return static_cast<int>(((u + 1) * static_cast<long long>(G) - 1) / U);
+}
+
+__device__ __forceinline__ void record_timeout(int* status, volatile int* abort_flag) {
+  atomicExch(status, kStatusTimeout);
+  *abort_flag = 1;
+}
+
+__device__ __forceinline__ float sumsq_bf16x8(uint4 v) {
+  float a = bf16_lo(v.x), b = bf16_hi(v.x), c = bf16_lo(v.y), d = bf16_hi(v.y);
+  float e = bf16_lo(v.z), f = bf16_hi(v.z), g = bf16_lo(v.w), h = bf16_hi(v.w);
+  float s0 = a * a, s1 = b * b;
+  s0 = fmaf(c, c, s0);
+  s1 = fmaf(d, d, s1);
+  s0 = fmaf(e, e, s0);
+  s1 = fmaf(f, f, s1);
+  s0 = fmaf(g, g, s0);
+  s1 = fmaf(h, h, s1);
+  return s0 + s1;
+}
+
+__device__ __forceinline__ float dot_bf16x8(uint4 w, const float* x) {
+  float s0 = bf16_lo(w.x) * x[0];
+  float s1 = bf16_hi(w.x) * x[1];
+  s0 = fmaf(bf16_lo(w.y), x[2], s0);
+  s1 = fmaf(bf16_hi(w.y), x[3], s1);
+  s0 = fmaf(bf16_lo(w.z), x[4], s0);
+  s1 = fmaf(bf16_hi(w.z), x[5], s1);
+  s0 = fmaf(bf16_lo(w.w), x[6], s0);
+  s1 = fmaf(bf16_hi(w.w), x[7], s1);
+  return s0 + s1;
+}
+
+// ===================================================================== norm
+__global__ void __launch_bounds__(kNormThreads, 1)
+    norm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA,
+                   const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmG,
+                   const NormArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  const uint32_t base_s = (raw_s + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base_s - raw_s);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + a.stages * a.stage_bytes);
+  uint64_t* empty = full + a.stages;
+  uint64_t* tmem_full = empty + a.stages;
+  uint64_t* tmem_empty = tmem_full + 1;
+  uint64_t* drain = tmem_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long U = a.units;
+  const int G = gridDim.x;
+  const long long u_begin = static_cast<long long>(blockIdx.x) * U / G;
+  const long long u_end = static_cast<long long>(blockIdx.x + 1) * U / G;
+  const int kb_total = a.kb_total;
+  const long long limit = a.wait_limit;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < a.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1 + 4);  // MMA commit + one arrive per epilogue warp
+    }
+    mbar_init(tmem_full, 1);
+    mbar_init(tmem_empty, 4);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmG);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, a.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t last_parity[kMaxStages];
+      int filled = 0;
+      for (long long u = u_begin; u < u_end; ++u) {
+        if (*abort_flag) break;
+        const int tc = static_cast<int>(u / kb_total);
+        const int kb = static_cast<int>(u % kb_total);
+        const int mt = tc / a.n_chunks;
+        const int ch = tc % a.n_chunks;
+        const int c0 = ch * a.chunk_n;
+        const int n_this = min(a.chunk_n, a.r - c0);
+        const int nboxes = (n_this + kBoxRows - 1) / kBoxRows;
+        if (!mbar_wait(&empty[stage], phase ^ 1u, limit)) {
+          record_timeout(a.status, abort_flag);
+          break;
+        }
+        mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(kBoxBytes * (1 + nboxes)));
+        const uint32_t sW = base_s + stage * a.stage_bytes;
+        const uint32_t sN = sW + kBoxBytes;
+        if (kb < a.kb_main) {
+          tma_load_2d(sW, &tmW, &full[stage], kb * kBK, mt * kBM);
+          for (int b = 0; b < nboxes; ++b) tma_load_2d(sN + b * kBoxBytes, &tmA, &full[stage], kb * kBK, c0 + b * kBoxRows);
+        } else {
+          const int e = kb - a.kb_main;
+          tma_load_2d(sW, &tmB, &full[stage], e * kBK, mt * kBM);
+          for (int b = 0; b < nboxes; ++b) tma_load_2d(sN + b * kBoxBytes, &tmG, &full[stage], e * kBK, c0 + b * kBoxRows);
+        }
+        last_parity[stage] = phase;
+        if (filled < a.stages) ++filled;
+        if (++stage == a.stages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      // Never leave a TMA copy in flight: wait for the latest fill of every stage.
+      for (int s = 0; s < filled; ++s) mbar_wait(&full[s], last_parity[s], limit);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int seg = 0;
+      for (long long u = u_begin; u < u_end; ++u) {
+        if (*abort_flag) break;
+        const int tc = static_cast<int>(u / kb_total);
+        const int kb = static_cast<int>(u % kb_total);
+        const int ch = tc % a.n_chunks;
+        const int n_this = min(a.chunk_n, a.r - ch * a.chunk_n);
+        const bool seg_first = (u == u_begin) || kb == 0;
+        const bool seg_last = (u == u_end - 1) || kb == kb_total - 1;
+        if (seg_first && seg > 0) {
+          if (!mbar_wait(tmem_empty, static_cast<uint32_t>((seg - 1) & 1), limit)) {
+            record_timeout(a.status, abort_flag);
+            break;
+          }
+          tc_fence_after();
+        }
+        if (!mbar_wait(&full[stage], phase, limit)) {
+          record_timeout(a.status, abort_flag);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sW = base_s + stage * a.stage_bytes;
+        const uint32_t sN = sW + kBoxBytes;
+#pragma unroll
+        for (int k = 0; k < kBK / 16; ++k) {
+          const uint64_t adesc = sw128_kmajor_desc(sW + k * 32);
+          for (int p = 0; p * 256 < n_this; ++p) {
+            const int pn = min(256, n_this - p * 256);
+            const uint64_t bdesc = sw128_kmajor_desc(sN + p * 256 * 128 + k * 32);
+            mma_bf16(tmem + p * 256, adesc, bdesc, idesc_bf16_f32(kBM, pn), (seg_first && k == 0) ? 0u : 1u);
+          }
+        }
+        mma_commit(&empty[stage]);
+        if (seg_last) {
+          mma_commit(tmem_full);
+          ++seg;
+        }
+        if (++stage == a.stages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      mma_commit(drain);
+      mbar_wait(drain, 0, limit);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row_local = q * 32 + lane;
+    const uint32_t tmem_lane = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    int stage = 0;
+    uint32_t phase = 0;
+    int seg = 0;
+    float base_acc = 0.f;
+    for (long long u = u_begin; u < u_end; ++u) {
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+      const int tc = static_cast<int>(u / kb_total);
+      const int kb = static_cast<int>(u % kb_total);
+      const int mt = tc / a.n_chunks;
+      const int ch = tc % a.n_chunks;
+      const int c0 = ch * a.chunk_n;
+      const int n_this = min(a.chunk_n, a.r - c0);
+      const bool seg_last = (u == u_end - 1) || kb == kb_total - 1;
+      if (!mbar_wait_warp(&full[stage], phase, limit)) {
+        if (lane == 0) record_timeout(a.status, abort_flag);
+        break;
+      }
+      if (ch == 0 && kb < a.kb_main) {
+        // ||W_i||^2 from the swizzled W stage: the 128-byte row of row_local
+        // holds its 64 K values with 16-byte chunks permuted; the sum does
+        // not care about the order, and visiting chunk (j ^ row % 8) keeps the
+        // eight rows of a quarter-warp on distinct banks.
+        const uint8_t* rowp = smem + stage * a.stage_bytes + row_local * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint4 v = *reinterpret_cast<const uint4*>(rowp + ((j ^ (row_local & 7)) << 4));
+          base_acc += sumsq_bf16x8(v);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);
+      if (++stage == a.stages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+      if (!seg_last) continue;
+
+      // ---- segment epilogue: <B_i, V_i> over this chunk's columns
+      if (!mbar_wait_warp(tmem_full, static_cast<uint32_t>(seg & 1), limit)) {
+        if (lane == 0) record_timeout(a.status, abort_flag);
+        break;
+      }
+      tc_fence_after();
+      const int row = mt * kBM + row_local;
+      const bool row_ok = row < a.d_out;
+      const __nv_bfloat16* brow = a.B + static_cast<size_t>(row_ok ? row : 0) * a.r + c0;
+      float dot = 0.f;
+      for (int j0 = 0; j0 < n_this; j0 += 32) {
+        float acc[32];
+        tmem_ld32(tmem_lane + j0, acc);
+        if (row_ok) {
+          const uint4* bp = reinterpret_cast<const uint4*>(brow + j0);
+          const int nv = min(4, (n_this - j0) >> 3);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            if (v < nv) dot += dot_bf16x8(__ldg(bp + v), acc + 8 * v);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tmem_empty);
+      ++seg;
+
+      const float partial = base_acc + a.two_s * dot;
+      base_acc = 0.f;
+      a.partials[static_cast<size_t>(blockIdx.x + tc) * kBM + row_local] = partial;
+
+      // ---- the last of the M tile's segment-warps to arrive finishes the tile
+      __threadfence();
+      __syncwarp();
+      int expected = 0;
+      for (int c2 = 0; c2 < a.n_chunks; ++c2) {
+        const long long s0 = static_cast<long long>(mt * a.n_chunks + c2) * kb_total;
+        expected += stream_k_owner(s0 + kb_total - 1, U, G) - stream_k_owner(s0, U, G) + 1;
+      }
+      int last = 0;
+      if (lane == 0) last = (atomicAdd(&a.counters[mt], 1) == 4 * expected - 1);
+      last = __shfl_sync(0xffffffffu, last, 0);
+      if (last) {
+        __threadfence();
+        for (int rr = lane; rr < kBM; rr += 32) {
+          float total = 0.f;
+          for (int c2 = 0; c2 < a.n_chunks; ++c2) {
+            const int tc2 = mt * a.n_chunks + c2;
+            const long long s0 = static_cast<long long>(tc2) * kb_total;
+            const int o0 = stream_k_owner(s0, U, G);
+            const int o1 = stream_k_owner(s0 + kb_total - 1, U, G);
+            for (int o = o0; o <= o1; ++o) total += ld_cg_f32(&a.partials[static_cast<size_t>(o + tc2) * kBM + rr]);
+          }
+          const int row2 = mt * kBM + rr;
+          if (row2 < a.d_out) a.n_out[row2] = sqrtf(fmaxf(total, 0.f));
+        }
+        if (lane == 0) a.counters[mt] = 0;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, a.tmem_cols);
+}
+
+// ===================================================================== Gram
+struct GramArgs {
+  int r, kb_main, splits, n_tiles;
+  long long wait_limit;
+  float* partial;  // [splits][tri tiles][128][128] fp32, upper-triangular tiles (mi <= ni) packed
+  int* status;
+};
+
+// Index of upper-triangular tile (mi <= ni) among nt x nt tiles, row-major.
+__host__ __device__ __forceinline__ int tri_index(int mi, int ni, int nt) {
+  return mi * nt - mi * (mi - 1) / 2 + (ni - mi);
+}
+
+constexpr int kGramStages = 4;
+constexpr uint32_t kGramStageBytes = 2 * kBoxBytes;
+
+__global__ void __launch_bounds__(kNormThreads, 1)
+    gram_tc_kernel(const __grid_constant__ CUtensorMap tmA, const GramArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  const uint32_t base_s = (raw_s + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base_s - raw_s);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kGramStages * kGramStageBytes);
+  uint64_t* empty = full + kGramStages;
+  uint64_t* tmem_full = empty + kGramStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long limit = a.wait_limit;
+
+  // (upper-triangular tile, K split) of this CTA
+  const int split = blockIdx.x % a.splits;
+  const int tile = blockIdx.x / a.splits;
+  const int n_tri = a.n_tiles * (a.n_tiles + 1) / 2;
+  int t = tile;
+  int mi = 0;
+  while (t >= a.n_tiles - mi) {
+    t -= a.n_tiles - mi;
+    ++mi;
+  }
+  const int ni = mi + t;
+  const int n_this = min(kBoxRows, a.r - ni * kBoxRows);
+  const int kb_lo = static_cast<int>(static_cast<long long>(split) * a.kb_main / a.splits);
+  const int kb_hi = static_cast<int>(static_cast<long long>(split + 1) * a.kb_main / a.splits);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kGramStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(tmem_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) tma_prefetch_desc(&tmA);
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t last_parity[kGramStages];
+      int filled = 0;
+      for (int kb = kb_lo; kb < kb_hi; ++kb) {
+        if (*abort_flag) break;
+        if (!mbar_wait(&empty[stage], phase ^ 1u, limit)) {
+          record_timeout(a.status, abort_flag);
+          break;
+        }
+        mbar_arrive_expect_tx(&full[stage], 2 * kBoxBytes);
+        const uint32_t sM = base_s + stage * kGramStageBytes;
+        tma_load_2d(sM, &tmA, &full[stage], kb * kBK, mi * kBoxRows);
+        tma_load_2d(sM + kBoxBytes, &tmA, &full[stage], kb * kBK, ni * kBoxRows);
+        last_parity[stage] = phase;
+        if (filled < kGramStages) ++filled;
+        if (++stage == kGramStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      for (int s = 0; s < filled; ++s) mbar_wait(&full[s], last_parity[s], limit);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int kb = kb_lo; kb < kb_hi; ++kb) {
+        if (*abort_flag) break;
+        if (!mbar_wait(&full[stage], phase, limit)) {
+          record_timeout(a.status, abort_flag);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sM = base_s + stage * kGramStageBytes;
+#pragma unroll
+        for (int k = 0; k < kBK / 16; ++k) {
+          mma_bf16(tmem, sw128_kmajor_desc(sM + k * 32), sw128_kmajor_desc(sM + kBoxBytes + k * 32),
+                   idesc_bf16_f32(kBM, n_this), (kb == kb_lo && k == 0) ? 0u : 1u);
+        }
+        mma_commit(&empty[stage]);
+        if (++stage == kGramStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      mma_commit(tmem_full);
+      mbar_wait(tmem_full, 0, limit);
+    }
+  } else {
+    const int q = warp & 3;
+    const int row_local = q * 32 + lane;
+    const int row = mi * kBoxRows + row_local;
+    const bool ok = mbar_wait_warp(tmem_full, 0, limit);
+    if (ok && !__any_sync(0xffffffffu, *abort_flag != 0)) {
+      tc_fence_after();
+      float* dst = a.partial + (static_cast<size_t>(split) * n_tri + tile) * (kBoxRows * kBoxRows) +
+                   static_cast<size_t>(row_local) * kBoxRows;
+      for (int j0 = 0; j0 < n_this; j0 += 32) {
+        float acc[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + j0, acc);
+        if (row < a.r) {
+          const int nv = min(8, (n_this - j0) >> 2);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            if (v < nv)
+              reinterpret_cast<float4*>(dst + j0)[v] =
+                  make_float4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
+        }
+      }
+    } else if (!ok && lane == 0) {
+      record_timeout(a.status, abort_flag);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 128);
+}
+
+// Sums the K splits of G = A A^T in fixed order, scales by s/2 and writes the
+// bf16 G' the norm kernel's K extension reads; also zeroes the norm kernel's
+// tile counters.
+__global__ void gram_reduce_kernel(const float* __restrict__ partial, int splits, int r, float half_s,
+                                   __nv_bfloat16* __restrict__ Gs, int* counters, int n_counters) {
+  const long long total = static_cast<long long>(r) * r;
+  const int nt = (r + kBoxRows - 1) / kBoxRows;
+  const long long split_stride = static_cast<long long>(nt * (nt + 1) / 2) * kBoxRows * kBoxRows;
+  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int j = static_cast<int>(idx / r);
+    const int k = static_cast<int>(idx % r);
+    const bool upper = (j / kBoxRows) <= (k / kBoxRows);
+    const int rr = upper ? j : k, cc = upper ? k : j;  // element of the stored upper tile
+    const long long src = static_cast<long long>(tri_index(rr / kBoxRows, cc / kBoxRows, nt)) * kBoxRows * kBoxRows +
+                          static_cast<long long>(rr % kBoxRows) * kBoxRows + (cc % kBoxRows);
+    float sum = 0.f;
+    for (int s = 0; s < splits; ++s) sum += partial[s * split_stride + src];
+    Gs[idx] = __float2bfloat16_rn(half_s * sum);
+  }
+  const int tid = blockIdx.x * blockDim.x + threadIdx.x;
+  if (tid < n_counters) counters[tid] = 0;
+}
+
+}  // namespace dora

@@ -1,0 +1,201 @@
+"""Thin Python binding of libdora.so (the C ABI in include/dora.h).
+
+The functions keep the C names.  They only marshal arguments: check dtypes,
+shapes and devices of torch tensors, take their data pointers and the current
+CUDA stream, allocate outputs / workspaces with torch when the caller passes
+none, and raise ``DoraError`` on a non-zero status.  Every step of the
+computation runs in libdora.so's CUDA kernels; there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdora.so")
+
+DORA_BF16 = 0
+DORA_F32 = 1
+
+DORA_OK = 0
+DORA_ERR_INVALID_ARG = 1
+DORA_ERR_UNSUPPORTED = 2
+DORA_ERR_WORKSPACE = 3
+DORA_ERR_CUDA = 4
+DORA_ERR_TIMEOUT = 5
+
+# every symbol include/dora.h declares, with its ctypes signature
+_c_void_p, _i64, _f32, _size = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "dora_factored_norm_workspace_size": (_size, [_i64, _i64, _i64, ctypes.c_int]),
+    "dora_factored_norm": (
+        ctypes.c_int,
+        [_c_void_p, _c_void_p, _c_void_p, _i64, _i64, _i64, _f32, ctypes.c_int, _c_void_p, _c_void_p, _size, _c_void_p],
+    ),
+    "dora_compose_fwd": (
+        ctypes.c_int,
+        [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _f32, _i64, _i64, ctypes.c_int, _c_void_p, _c_void_p],
+    ),
+    "dora_compose_bwd_workspace_size": (_size, [_i64, _i64]),
+    "dora_compose_bwd": (
+        ctypes.c_int,
+        [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _f32, _i64, _i64, ctypes.c_int,
+         _c_void_p, _c_void_p, _c_void_p, _c_void_p, _size, _c_void_p],
+    ),
+    "dora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "dora_device_status": (ctypes.c_int, [_c_void_p]),
+    "dora_num_sms": (ctypes.c_int, []),
+}
+
+_lib = None
+
+
+class DoraError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libdora.so (built in-tree); raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m factored_weight_norm_b200.build` "
+                "(nvcc, sm_100a). There is no CPU or PyTorch fallback."
+            )
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().dora_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != DORA_OK:
+        raise DoraError(status, where)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return DORA_BF16
+    if t.dtype == torch.float32:
+        return DORA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}: bf16 or fp32 only")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dense_cuda(*ts):
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("tensors must live on a CUDA device")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous (row-major)")
+
+
+# ---------------------------------------------------------------- C names
+def dora_factored_norm_workspace_size(d_out: int, d_in: int, r: int, dtype: torch.dtype = torch.bfloat16) -> int:
+    return int(lib().dora_factored_norm_workspace_size(d_out, d_in, r, _dt(torch.empty(0, dtype=dtype))))
+
+
+def dora_compose_bwd_workspace_size(tokens: int, d_out: int) -> int:
+    return int(lib().dora_compose_bwd_workspace_size(tokens, d_out))
+
+
+def dora_num_sms() -> int:
+    return int(lib().dora_num_sms())
+
+
+def dora_device_status(stream=None) -> int:
+    return int(lib().dora_device_status(_stream(stream)))
+
+
+def dora_status_string(status: int) -> str:
+    return status_string(status)
+
+
+def dora_factored_norm(W, A, B, s: float, n_out=None, workspace=None, stream=None):
+    """n = ||W + s B A||_row as fp32 [d_out] (factored; no dense B A)."""
+    _dense_cuda(W, A, B, n_out, workspace)
+    d_out, d_in = W.shape
+    r = A.shape[0]
+    if A.shape != (r, d_in) or B.shape != (d_out, r):
+        raise ValueError(f"shape mismatch: W {tuple(W.shape)}, A {tuple(A.shape)}, B {tuple(B.shape)}")
+    if not (W.dtype == A.dtype == B.dtype):
+        raise TypeError("W, A and B must share one dtype")
+    if n_out is None:
+        n_out = torch.empty(d_out, dtype=torch.float32, device=W.device)
+    need = dora_factored_norm_workspace_size(d_out, d_in, r, W.dtype)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
+    st = lib().dora_factored_norm(
+        _ptr(W), _ptr(A), _ptr(B), d_out, d_in, r, float(s), _dt(W), _ptr(n_out),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream),
+    )
+    _check(st, "dora_factored_norm")
+    return n_out
+
+
+def dora_compose_fwd(base_out, lora_out, m, n, s: float, y=None, stream=None):
+    """y = (m / n) * (base_out + s * lora_out), single fused pass."""
+    _dense_cuda(base_out, lora_out, m, n, y)
+    tokens, d_out = base_out.shape
+    if lora_out.shape != base_out.shape or m.shape != (d_out,) or n.shape != (d_out,):
+        raise ValueError("shape mismatch in dora_compose_fwd")
+    if m.dtype != torch.float32 or n.dtype != torch.float32:
+        raise TypeError("m and n must be fp32")
+    if y is None:
+        y = torch.empty_like(base_out)
+    st = lib().dora_compose_fwd(
+        _ptr(base_out), _ptr(lora_out), _ptr(m), _ptr(n), float(s), tokens, d_out, _dt(base_out), _ptr(y),
+        _stream(stream),
+    )
+    _check(st, "dora_compose_fwd")
+    return y
+
+
+def dora_compose_bwd(dy, base_out, lora_out, m, n, s: float, d_base=None, d_lora=None, d_m=None, workspace=None,
+                     stream=None):
+    """(d_base, d_lora, d_m) of the compose with n held constant."""
+    _dense_cuda(dy, base_out, lora_out, m, n, d_base, d_lora, d_m, workspace)
+    tokens, d_out = base_out.shape
+    if dy.shape != base_out.shape or lora_out.shape != base_out.shape:
+        raise ValueError("shape mismatch in dora_compose_bwd")
+    if m.dtype != torch.float32 or n.dtype != torch.float32:
+        raise TypeError("m and n must be fp32")
+    if d_base is None:
+        d_base = torch.empty_like(base_out)
+    if d_lora is None:
+        d_lora = torch.empty_like(base_out)
+    if d_m is None:
+        d_m = torch.empty(d_out, dtype=torch.float32, device=base_out.device)
+    need = dora_compose_bwd_workspace_size(tokens, d_out)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=base_out.device)
+    st = lib().dora_compose_bwd(
+        _ptr(dy), _ptr(base_out), _ptr(lora_out), _ptr(m), _ptr(n), float(s), tokens, d_out, _dt(base_out),
+        _ptr(d_base), _ptr(d_lora), _ptr(d_m), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream),
+    )
+    _check(st, "dora_compose_bwd")
+    return d_base, d_lora, d_m

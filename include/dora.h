@@ -1,0 +1,122 @@
+/*
+ * dora.h - C ABI of the B200 (sm_100a) DoRA factored-norm / fused-compose library.
+ *
+ * Method: "Scaling DoRA: High-Rank Adaptation via Factored Norms and Fused
+ * Kernels" (Zelenin & Zhuravlyova, arXiv 2603.22276), Abstract.  DoRA writes
+ * the adapted weight as W' = m * (W + s B A) / ||W + s B A||_row.  The row norm
+ * is computed from base, cross and Gram terms without forming B A, and the
+ * magnitude rescaling is composed with the base and LoRA outputs in one pass.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Layout: dense, row-major, contiguous.  W is [d_out, d_in] (frozen base
+ *    weight), A is [r, d_in] (lora_A), B is [d_out, r] (lora_B), activations
+ *    base_out / lora_out / dy / y / d_base / d_lora are [tokens, d_out].
+ *    lora_out is UNSCALED (x A^T B^T); the scaling s is applied here.
+ *  - dtype: DORA_BF16 or DORA_F32 applies to W, A, B and the activations.
+ *    m, n and d_m are always fp32 [d_out].
+ *  - Pointers are device pointers unless stated.  The caller owns and allocates
+ *    every buffer, including the workspace; the library never allocates device
+ *    memory, so no O(d_out * d_in) temporary ever exists.
+ *  - bf16 requires 16-byte aligned pointers, d_in and d_out multiples of 8 and
+ *    r a multiple of 16 (else DORA_ERR_UNSUPPORTED).  fp32 accepts any shape
+ *    with 4-byte aligned pointers.
+ *  - stream is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Every call is asynchronous on it and returns once the work is enqueued.
+ *  - Errors: argument errors are detected on the host before anything is
+ *    launched and return DORA_ERR_INVALID_ARG / DORA_ERR_UNSUPPORTED /
+ *    DORA_ERR_WORKSPACE.  A failed launch returns DORA_ERR_CUDA.  Kernels that
+ *    wait on other threads bound every wait; if one gives up it records
+ *    DORA_ERR_TIMEOUT in a device-side word that dora_device_status() reports.
+ *  - Outputs are overwritten, never accumulated into.  Results are
+ *    deterministic: every reduction runs in a fixed order.
+ */
+#ifndef DORA_H_
+#define DORA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DORA_API __attribute__((visibility("default")))
+#else
+#define DORA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { DORA_BF16 = 0, DORA_F32 = 1 } dora_dtype;
+
+typedef enum {
+  DORA_OK = 0,
+  DORA_ERR_INVALID_ARG = 1, /* null pointer, negative size, r > d_in ... */
+  DORA_ERR_UNSUPPORTED = 2, /* alignment / shape / dtype this build does not handle */
+  DORA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than the size query */
+  DORA_ERR_CUDA = 4,        /* a CUDA runtime call failed (launch, attribute ...) */
+  DORA_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up */
+} dora_status;
+
+/* Bytes of workspace dora_factored_norm needs for this shape (0 never means
+ * "no workspace" for valid shapes; returns 0 for invalid shapes). */
+DORA_API size_t dora_factored_norm_workspace_size(int64_t d_out, int64_t d_in, int64_t r, dora_dtype dt);
+
+/* Factored row norm of W + s B A (Scaling DoRA, Abstract: "base, cross, and
+ * Gram terms computable through O(d_out r + r^2) intermediates"):
+ *
+ *   n_i = sqrt(max(||W_i||^2 + 2 s <B_i, (W A^T)_i> + s^2 B_i (A A^T) B_i^T, 0))
+ *
+ * n_out: fp32 [d_out], overwritten.  workspace: device buffer of at least
+ * dora_factored_norm_workspace_size() bytes, 256-byte aligned, contents
+ * ignored on entry and clobbered; it is O(d_out r + r^2 + SMs * 128) and never
+ * O(d_out d_in).  r == 0 or s == 0 give the plain row norm of W.  bf16: W is
+ * streamed from HBM once by tcgen05 tensor-core GEMM tiles; fp32: CUDA-core
+ * fp32 arithmetic (no TF32). */
+DORA_API int dora_factored_norm(const void* W, const void* A, const void* B, int64_t d_out, int64_t d_in, int64_t r,
+                       float s, dora_dtype dt, float* n_out, void* workspace, size_t workspace_bytes,
+                       void* stream);
+
+/* Fused DoRA compose, one pass (Scaling DoRA, Abstract: the four-kernel
+ * composition collapsed into a single pass, in a numerically stable form for
+ * the near-unity regime):
+ *
+ *   g = m / n,  delta = (m - n) / n            (fp32, per output channel)
+ *   y = base + (delta * base + g * s * lora)   (fp32 arithmetic, one rounding)
+ *
+ * which equals g * (base + s * lora) without rounding g or g - 1 to the
+ * activation type.  tokens may be 0 (nothing is launched). */
+DORA_API int dora_compose_fwd(const void* base_out, const void* lora_out, const float* m, const float* n, float s,
+                     int64_t tokens, int64_t d_out, dora_dtype dt, void* y, void* stream);
+
+/* Bytes of workspace dora_compose_bwd needs (column partial sums). */
+DORA_API size_t dora_compose_bwd_workspace_size(int64_t tokens, int64_t d_out);
+
+/* Backward of dora_compose_fwd with n held constant (the norm is detached):
+ *
+ *   d_base = g * dy,   d_lora = s * g * dy,
+ *   d_m_i  = (sum_t dy[t,i] * (base[t,i] + s * lora[t,i])) / n_i
+ *
+ * d_base, d_lora: [tokens, d_out] in dt, overwritten.  d_m: fp32 [d_out],
+ * overwritten (tokens == 0 gives d_m = 0).  The token reduction accumulates
+ * in fp32 and combines per-chunk partials in a fixed order. */
+DORA_API int dora_compose_bwd(const void* dy, const void* base_out, const void* lora_out, const float* m, const float* n,
+                     float s, int64_t tokens, int64_t d_out, dora_dtype dt, void* d_base, void* d_lora, float* d_m,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* Human-readable name of a dora_status value (static storage). */
+DORA_API const char* dora_status_string(int status);
+
+/* Reads and clears the device-side status word of the current device
+ * (DORA_OK or DORA_ERR_TIMEOUT).  Synchronises `stream` first. */
+DORA_API int dora_device_status(void* stream);
+
+/* Number of SMs the persistent kernels size their grids to on the current
+ * device (the grid is a multiple of this count).  Returns 0 when no device. */
+DORA_API int dora_num_sms(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DORA_H_ */

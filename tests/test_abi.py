@@ -1,0 +1,148 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared
+symbol, validates arguments before touching the GPU, and sizes workspaces
+without any O(d_out * d_in) term.  No compute call is made here."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from factored_weight_norm_b200 import build as build_mod
+from factored_weight_norm_b200 import dora as D
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dora.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return D.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dora_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("dora_factored_norm", "dora_compose_fwd", "dora_compose_bwd"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    out = subprocess.run(["nm", "-D", "--defined-only", D.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (dora_[a-z0-9_]+)", out))
+    missing = [n for n in names if n not in exported]
+    assert not missing, f"declared but not exported: {missing}"
+    extra = sorted(exported - set(names))
+    assert not extra, f"exported but not declared: {extra}"
+    assert set(D.SIGNATURES) == set(names)
+
+
+def test_status_strings(lib):
+    for st in range(6):
+        assert D.status_string(st).startswith("DORA_")
+    assert "unknown" in D.status_string(99)
+
+
+FAKE = ctypes.c_void_p(0x10000)      # 64 KiB aligned, never dereferenced
+MISALIGNED = ctypes.c_void_p(0x10002)
+
+
+def _norm(lib, W=FAKE, A=FAKE, B=FAKE, d_out=64, d_in=128, r=16, dt=D.DORA_BF16, n=FAKE, ws=FAKE, wsb=1 << 30):
+    return lib.dora_factored_norm(W, A, B, d_out, d_in, r, 0.5, dt, n, ws, wsb, None)
+
+
+def test_norm_argument_errors(lib):
+    assert _norm(lib, W=None) == D.DORA_ERR_INVALID_ARG
+    assert _norm(lib, n=None) == D.DORA_ERR_INVALID_ARG
+    assert _norm(lib, A=None) == D.DORA_ERR_INVALID_ARG
+    assert _norm(lib, d_out=-1) == D.DORA_ERR_INVALID_ARG
+    assert _norm(lib, r=-3) == D.DORA_ERR_INVALID_ARG
+    assert _norm(lib, dt=7) == D.DORA_ERR_UNSUPPORTED
+    assert _norm(lib, d_in=100) == D.DORA_ERR_UNSUPPORTED  # bf16 needs d_in % 8 == 0
+    assert _norm(lib, r=24) == D.DORA_ERR_UNSUPPORTED      # bf16 needs r % 16 == 0
+    assert _norm(lib, r=8192) == D.DORA_ERR_UNSUPPORTED    # beyond the supported rank
+    assert _norm(lib, W=MISALIGNED) == D.DORA_ERR_UNSUPPORTED
+    assert _norm(lib, ws=None) == D.DORA_ERR_WORKSPACE
+    assert _norm(lib, wsb=16) == D.DORA_ERR_WORKSPACE
+    assert _norm(lib, ws=MISALIGNED) == D.DORA_ERR_UNSUPPORTED
+    assert _norm(lib, d_out=0) == D.DORA_OK  # nothing to do, nothing launched
+
+
+def test_compose_argument_errors(lib):
+    f = lib.dora_compose_fwd
+    assert f(None, FAKE, FAKE, FAKE, 0.5, 4, 64, D.DORA_BF16, FAKE, None) == D.DORA_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, FAKE, 0.5, -1, 64, D.DORA_BF16, FAKE, None) == D.DORA_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, FAKE, 0.5, 4, 60, D.DORA_BF16, FAKE, None) == D.DORA_ERR_UNSUPPORTED
+    assert f(FAKE, MISALIGNED, FAKE, FAKE, 0.5, 4, 64, D.DORA_BF16, FAKE, None) == D.DORA_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, FAKE, 0.5, 0, 64, D.DORA_BF16, FAKE, None) == D.DORA_OK
+    b = lib.dora_compose_bwd
+    ws = lib.dora_compose_bwd_workspace_size(4, 64)
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, 0.5, 4, 64, D.DORA_BF16, FAKE, FAKE, FAKE, FAKE, ws, None]
+    bad = list(args)
+    bad[11] = None  # d_m
+    assert b(*bad) == D.DORA_ERR_INVALID_ARG
+    bad = list(args)
+    bad[13] = ws - 1
+    assert b(*bad) == D.DORA_ERR_WORKSPACE
+    bad = list(args)
+    bad[12] = None
+    assert b(*bad) == D.DORA_ERR_WORKSPACE
+    bad = list(args)
+    bad[7] = 12
+    assert b(*bad) == D.DORA_ERR_UNSUPPORTED
+
+
+def test_workspace_has_no_dense_term(lib):
+    # the dense product B A would be d_out * d_in * 2 bytes; the workspace is
+    # O(d_out r + r^2 + SMs * 128)
+    for d_out, d_in, r in ((8192, 8192, 384), (27648, 5120, 384), (8192, 8192, 768), (4096, 4096, 64)):
+        ws = lib.dora_factored_norm_workspace_size(d_out, d_in, r, D.DORA_BF16)
+        assert 0 < ws < d_out * d_in * 2 / 8, (d_out, d_in, r, ws)
+        # growing d_in does not grow the workspace
+        assert lib.dora_factored_norm_workspace_size(d_out, 4 * d_in, r, D.DORA_BF16) == ws
+    ws_bwd = lib.dora_compose_bwd_workspace_size(8192, 8192)
+    assert 0 < ws_bwd < 8192 * 8192 * 2 / 16
+    assert lib.dora_compose_bwd_workspace_size(65536, 8192) == ws_bwd  # independent of tokens
+    assert lib.dora_factored_norm_workspace_size(-1, 8, 16, D.DORA_BF16) == 0
+
+
+def test_num_sms_without_device(lib):
+    import torch
+
+    if not torch.cuda.is_available():
+        assert lib.dora_num_sms() == 0
+
+
+# ------------------------------------------------ stream-K schedule algebra
+def _owner(u, U, G):
+    return ((u + 1) * G - 1) // U
+
+
+@pytest.mark.parametrize("U,G", [(1, 1), (3, 3), (7, 3), (8384, 148), (134 * 216, 148), (10, 7)])
+def test_stream_k_partition(U, G):
+    """Ranges [floor(cU/G), floor((c+1)U/G)) tile [0, U); owner() inverts them;
+    segment index c + tc is unique when segments split at tile boundaries."""
+    ranges = [(c * U // G, (c + 1) * U // G) for c in range(G)]
+    assert ranges[0][0] == 0 and ranges[-1][1] == U
+    for (a0, a1), (b0, b1) in zip(ranges, ranges[1:]):
+        assert a1 == b0
+    for c, (a, b) in enumerate(ranges):
+        for u in range(a, b):
+            assert _owner(u, U, G) == c
+    for kb_total in (1, 3, 134):
+        seen = set()
+        for c, (a, b) in enumerate(ranges):
+            for u in range(a, b):
+                if u == a or u % kb_total == 0:
+                    idx = c + u // kb_total
+                    assert idx not in seen
+                    seen.add(idx)
+        assert max(seen, default=0) < G + (U + kb_total - 1) // kb_total
