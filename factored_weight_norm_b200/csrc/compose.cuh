@@ -76,7 +76,7 @@ struct VecIO<float, 1> {
 
 // ------------------------------------------------------------------ forward
 template <typename T, int VEC>
-__global__ void __launch_bounds__(256) compose_fwd_kernel(const T* __restrict__ base, const T* __restrict__ lora,
+__global__ void __launch_bounds__(256, 3) compose_fwd_kernel(const T* __restrict__ base, const T* __restrict__ lora,
                                                           const float* __restrict__ m,
                                                           const float* __restrict__ n, float s,
                                                           long long tokens, long long nvec, long long d_out,
@@ -126,7 +126,7 @@ constexpr int kBwdVecs = 16;      // vectors (column groups) per CTA strip
 constexpr int kBwdSlots = 16;     // rows visited concurrently by one CTA
 
 template <typename T, int VEC>
-__global__ void __launch_bounds__(kBwdThreads) compose_bwd_kernel(
+__global__ void __launch_bounds__(kBwdThreads, 3) compose_bwd_kernel(
     const T* __restrict__ dy, const T* __restrict__ base, const T* __restrict__ lora, const float* __restrict__ m,
     const float* __restrict__ n, float s, long long tokens, long long nvec, long long d_out, T* __restrict__ d_base,
     T* __restrict__ d_lora, float* __restrict__ partial, int* __restrict__ counters, float* __restrict__ d_m,

@@ -31,7 +31,6 @@ constexpr long long kWaitLimitCycles = 2000000000LL;  // ~1 s at B200 clocks
 constexpr int kMaxGrid = 1024;                         // bound on the persistent grid
 constexpr int kMaxGramSplits = 32;
 constexpr int kMaxBwdChunks = 64;
-constexpr int kCtasPerSm = 8;  // 256-thread CTAs that fill an SM's 2048 thread slots
 constexpr int kMaxDevices = 64;
 constexpr int64_t kMaxRank = 4096;
 
@@ -117,7 +116,7 @@ TcPlan plan_tc(int64_t d_out, int64_t d_in, int64_t r) {
   p.kb_total = p.kb_main + p.kb_ext;
   p.units = static_cast<long long>(p.m_tiles) * p.n_chunks * p.kb_total;
   const int nt = static_cast<int>(cdiv(r, kBoxRows));
-  p.gram_tiles = nt * (nt + 1) / 2;
+  p.gram_tiles = nt * nt;
   p.gram_splits_max = std::max(1, std::min({kMaxGramSplits, 160 / p.gram_tiles, p.kb_main}));
   size_t off = 0;
   p.off_gs = off;
@@ -136,6 +135,35 @@ size_t f32_norm_ws(int64_t r) { return align_up(static_cast<size_t>(r) * r * 4, 
 
 int launch_error() { return cudaGetLastError() == cudaSuccess ? DORA_OK : DORA_ERR_CUDA; }
 
+// Resident CTAs per SM of a kernel at the given block size (at least 1).
+template <typename K>
+int ctas_per_sm(K kernel, int threads) {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, 0) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    return 1;
+  }
+  return n;
+}
+
+// Number of row chunks k in [1, k_max] for `cols` column strips that fills
+// whole waves of `slots` resident CTAs best (ties go to the smaller k).
+long long pick_chunks(long long cols, long long slots, long long k_max) {
+  long long best = 1;
+  double best_eff = -1.0;
+  for (long long k = 1; k <= std::max<long long>(1, k_max); ++k) {
+    const long long ctas = cols * k;
+    const long long waves = (ctas + slots - 1) / slots;
+    const double eff = static_cast<double>(ctas) / static_cast<double>(waves * slots);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = k;
+    }
+    if (waves > 4) break;
+  }
+  return best;
+}
+
 int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_t d_in, int64_t r, float s,
               float* n_out, void* ws, cudaStream_t st, DeviceInfo* dev) {
   const TcPlan p = plan_tc(d_out, d_in, r);
@@ -150,7 +178,10 @@ int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_
       make_map(&tmG, Gs, r, r))
     return DORA_ERR_CUDA;
 
-  // 1) Gram partial tiles, 2) reduce to bf16 (s/2) G and zero the counters
+  // 1) Gram partial tiles, 2) reduce to bf16 (s/2) G and zero the counters,
+  // 3) the persistent GEMM; 2) and 3) use programmatic dependent launch so
+  // they are scheduled while their predecessor still runs and wait for it
+  // only where they read its results.
   GramArgs ga{};
   ga.r = static_cast<int>(r);
   ga.kb_main = p.kb_main;
@@ -162,12 +193,23 @@ int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_
   const size_t gram_smem = kGramStages * kGramStageBytes + (2 * kGramStages + 1) * 8 + 16 + 1024;
   gram_tc_kernel<<<p.gram_tiles * ga.splits, kNormThreads, gram_smem, st>>>(tmA, ga);
   if (launch_error()) return DORA_ERR_CUDA;
-  const long long rr = static_cast<long long>(r) * r;
-  const int red_blocks = static_cast<int>(std::max<long long>(cdiv(p.m_tiles, 256), std::min<long long>(cdiv(rr, 256), 4 * dev->num_sms)));
-  gram_reduce_kernel<<<red_blocks, 256, 0, st>>>(Gp, ga.splits, static_cast<int>(r), 0.5f * s, Gs, cnt, p.m_tiles);
-  if (launch_error()) return DORA_ERR_CUDA;
 
-  // 3) persistent stream-K GEMM with the fused norm epilogue
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.stream = st;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+
+  const long long rr = static_cast<long long>(r) * r;
+  cfg.gridDim = dim3(static_cast<unsigned>(std::max<long long>(cdiv(p.m_tiles, 256), std::min<long long>(cdiv(rr, 256), 4 * dev->num_sms))));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  if (cudaLaunchKernelEx(&cfg, gram_reduce_kernel, static_cast<const float*>(Gp), ga.splits, static_cast<int>(r),
+                         0.5f * s, Gs, cnt, p.m_tiles) != cudaSuccess)
+    return DORA_ERR_CUDA;
+
   NormArgs na{};
   na.d_out = static_cast<int>(d_out);
   na.d_in = static_cast<int>(d_in);
@@ -178,8 +220,7 @@ int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_
   na.kb_main = p.kb_main;
   na.kb_total = p.kb_total;
   na.units = p.units;
-  na.n_tile_bytes = static_cast<uint32_t>(cdiv(p.chunk_n, kBoxRows) * kBoxBytes);
-  na.stage_bytes = kBoxBytes + na.n_tile_bytes;
+  na.stage_bytes = static_cast<uint32_t>(kBoxBytes * (1 + cdiv(p.chunk_n, kBoxRows)));
   const size_t fixed = 1024 + 64 + 16;
   na.stages = static_cast<int>(std::min<size_t>(kMaxStages, (dev->smem_optin - fixed) / (na.stage_bytes + 16)));
   if (na.stages < 2) return DORA_ERR_UNSUPPORTED;
@@ -188,14 +229,15 @@ int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_
   na.tmem_cols = cols;
   na.two_s = 2.0f * s;
   na.wait_limit = kWaitLimitCycles;
-  na.B = static_cast<const __nv_bfloat16*>(B);
   na.partials = part;
   na.counters = cnt;
   na.n_out = n_out;
   na.status = dev->status;
   const int grid = static_cast<int>(std::min<long long>({static_cast<long long>(dev->num_sms), p.units, kMaxGrid}));
-  const size_t smem = static_cast<size_t>(na.stages) * na.stage_bytes + (2 * na.stages + 3) * 8 + 16 + 1024;
-  norm_tc_kernel<<<grid, kNormThreads, smem, st>>>(tmW, tmA, tmB, tmG, na);
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kNormThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(na.stages) * na.stage_bytes + (2 * na.stages + 3) * 8 + 16 + 1024;
+  if (cudaLaunchKernelEx(&cfg, norm_tc_kernel, tmW, tmA, tmB, tmG, na) != cudaSuccess) return DORA_ERR_CUDA;
   return launch_error();
 }
 
@@ -296,7 +338,15 @@ int dora_compose_fwd(const void* base_out, const void* lora_out, const float* m,
   const int threads = static_cast<int>(std::min<long long>(256, align_up(static_cast<size_t>(nvec), 32)));
   const long long gx = cdiv(nvec, threads);
   if (gx > INT32_MAX) return DORA_ERR_UNSUPPORTED;
-  const long long gy = std::max<long long>(1, std::min<long long>({static_cast<long long>(dev->num_sms) * kCtasPerSm / gx, tokens, 65535}));
+  int occ = 1;
+  if (dt == DORA_BF16)
+    occ = ctas_per_sm(compose_fwd_kernel<__nv_bfloat16, 8>, threads);
+  else if (vec == 4)
+    occ = ctas_per_sm(compose_fwd_kernel<float, 4>, threads);
+  else
+    occ = ctas_per_sm(compose_fwd_kernel<float, 1>, threads);
+  const long long slots = static_cast<long long>(dev->num_sms) * occ;
+  const long long gy = pick_chunks(gx, slots, std::min<long long>(tokens, 65535));
   const long long rows = cdiv(tokens, gy);
   const long long gy2 = cdiv(tokens, rows);
   dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy2));
@@ -356,9 +406,15 @@ int dora_compose_bwd(const void* dy, const void* base_out, const void* lora_out,
   const long long nvec = d_out / vec;
   const long long strips = cdiv(nvec, kBwdVecs);
   if (strips > INT32_MAX) return DORA_ERR_UNSUPPORTED;
-  const long long chunks = std::max<long long>(
-      1, std::min<long long>({static_cast<long long>(dev->num_sms) * kCtasPerSm / strips, kMaxBwdChunks,
-                              cdiv(tokens, kBwdSlots)}));
+  int occ = 1;
+  if (dt == DORA_BF16)
+    occ = ctas_per_sm(compose_bwd_kernel<__nv_bfloat16, 8>, kBwdThreads);
+  else if (vec == 4)
+    occ = ctas_per_sm(compose_bwd_kernel<float, 4>, kBwdThreads);
+  else
+    occ = ctas_per_sm(compose_bwd_kernel<float, 1>, kBwdThreads);
+  const long long chunks = pick_chunks(strips, static_cast<long long>(dev->num_sms) * occ,
+                                       std::min<long long>(kMaxBwdChunks, cdiv(tokens, kBwdSlots)));
   const long long rows = cdiv(tokens, chunks);
   const long long chunks2 = cdiv(tokens, rows);
   uint8_t* w = static_cast<uint8_t*>(workspace);

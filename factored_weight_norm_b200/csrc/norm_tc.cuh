@@ -13,15 +13,19 @@
 // epilogue gives every term; W is streamed from HBM exactly once and the
 // [d_out, r] product V never leaves TMEM.
 //
-// Kernels:
-//   gram_tc_kernel     G = A A^T partial tiles (upper triangle, split over K)
+// Kernels (one stream, chained with programmatic dependent launch):
+//   gram_tc_kernel     G = A A^T as 128x128 tiles split over K (fp32 partials)
 //   gram_reduce_kernel sums the K splits in fixed order, writes bf16 G'
 //   norm_tc_kernel     persistent stream-K GEMM over (M tile, N chunk, K
-//                      block) units; each CTA owns a contiguous unit range.
-//                      Epilogue: ||W_i||^2 from the shared-memory W stages,
-//                      <B_i, V_i> from TMEM; per-(row, segment) scalar
-//                      partials; the last CTA to finish an M tile sums its
-//                      partials in fixed order and writes n = sqrt(max(., 0)).
+//                      block) units; each CTA owns a contiguous unit range and
+//                      starts streaming W before the Gram kernels finish (it
+//                      only waits for them before its first K-extension block).
+//                      Epilogue: ||W_i||^2 from the shared-memory W stages;
+//                      B's rows arrive through the same TMA ring after each
+//                      segment and are dotted with V_i read from TMEM; one
+//                      fp32 partial per (row, segment); the last warp to finish
+//                      an M tile sums its partials in fixed order and writes
+//                      n = sqrt(max(., 0)).
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -42,15 +46,13 @@ struct NormArgs {
   int m_tiles, n_chunks, chunk_n, kb_main, kb_total;
   long long units;
   int stages;
-  uint32_t stage_bytes;   // W-side tile + N-side tiles
-  uint32_t n_tile_bytes;  // bytes reserved for the N-side tiles of a stage
+  uint32_t stage_bytes;   // W-side tile + N-side tiles (a multiple of kBoxBytes)
   uint32_t tmem_cols;
   float two_s;
   long long wait_limit;
-  const __nv_bfloat16* B;  // [d_out, r], read by the epilogue
-  float* partials;         // [(gridDim.x + m_tiles * n_chunks) * 128]
-  int* counters;           // [m_tiles], zero on entry, left zero on exit
-  float* n_out;            // [d_out]
+  float* partials;        // [(gridDim.x + m_tiles * n_chunks) * 128]
+  int* counters;          // [m_tiles], zeroed by gram_reduce_kernel
+  float* n_out;           // [d_out]
   int* status;
 };
 
@@ -90,6 +92,55 @@ __device__ __forceinline__ float dot_bf16x8(uint4 w, const float* x) {
   return s0 + s1;
 }
 
+// Byte offset of 16-byte chunk `c` of row `row` inside a 128-byte-swizzled tile.
+__device__ __forceinline__ uint32_t sw128_chunk(int row, int c) {
+  return static_cast<uint32_t>(row * 128 + ((c ^ (row & 7)) << 4));
+}
+
+// Walks a CTA's contiguous range of (M tile, N chunk, K block) units in order.
+// Only the start needs a division; stepping is compare-and-increment, so the
+// single-thread producer and MMA loops spend a few instructions per unit.
+struct UnitIter {
+  int tc, kb, mt, ch, c0, n_this, left;
+  bool seg_first;
+
+  __device__ __forceinline__ void start(const NormArgs& a, long long u_begin, long long u_end) {
+    tc = static_cast<int>(u_begin / a.kb_total);
+    kb = static_cast<int>(u_begin - static_cast<long long>(tc) * a.kb_total);
+    mt = tc / a.n_chunks;
+    ch = tc - mt * a.n_chunks;
+    c0 = ch * a.chunk_n;
+    n_this = min(a.chunk_n, a.r - c0);
+    left = static_cast<int>(u_end - u_begin);
+    seg_first = true;
+  }
+  __device__ __forceinline__ bool valid() const { return left > 0; }
+  __device__ __forceinline__ bool seg_last(const NormArgs& a) const { return left == 1 || kb == a.kb_total - 1; }
+  __device__ __forceinline__ void next(const NormArgs& a) {
+    --left;
+    if (++kb == a.kb_total) {
+      kb = 0;
+      ++tc;
+      if (++ch == a.n_chunks) {
+        ch = 0;
+        ++mt;
+      }
+      c0 = ch * a.chunk_n;
+      n_this = min(a.chunk_n, a.r - c0);
+      seg_first = true;
+    } else {
+      seg_first = false;
+    }
+  }
+};
+
+// Ring slots that carry B's rows for a segment epilogue.
+__device__ __forceinline__ int b_stages(const NormArgs& a, int n_this) {
+  const int nbox = (n_this + kBK - 1) / kBK;
+  const int slots = static_cast<int>(a.stage_bytes / kBoxBytes);
+  return (nbox + slots - 1) / slots;
+}
+
 // ===================================================================== norm
 __global__ void __launch_bounds__(kNormThreads, 1)
     norm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA,
@@ -113,13 +164,13 @@ __global__ void __launch_bounds__(kNormThreads, 1)
   const int G = gridDim.x;
   const long long u_begin = static_cast<long long>(blockIdx.x) * U / G;
   const long long u_end = static_cast<long long>(blockIdx.x + 1) * U / G;
-  const int kb_total = a.kb_total;
   const long long limit = a.wait_limit;
+  const int slots = static_cast<int>(a.stage_bytes / kBoxBytes);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.stages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + 4);  // MMA commit + one arrive per epilogue warp
+      mbar_init(&empty[s], 1 + 4);  // MMA warp + one arrive per epilogue warp
     }
     mbar_init(tmem_full, 1);
     mbar_init(tmem_empty, 4);
@@ -144,90 +195,131 @@ __global__ void __launch_bounds__(kNormThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t last_parity[kMaxStages];
-      int filled = 0;
-      for (long long u = u_begin; u < u_end; ++u) {
-        if (*abort_flag) break;
-        const int tc = static_cast<int>(u / kb_total);
-        const int kb = static_cast<int>(u % kb_total);
-        const int mt = tc / a.n_chunks;
-        const int ch = tc % a.n_chunks;
-        const int c0 = ch * a.chunk_n;
-        const int n_this = min(a.chunk_n, a.r - c0);
-        const int nboxes = (n_this + kBoxRows - 1) / kBoxRows;
-        if (!mbar_wait(&empty[stage], phase ^ 1u, limit)) {
-          record_timeout(a.status, abort_flag);
-          break;
-        }
-        mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(kBoxBytes * (1 + nboxes)));
-        const uint32_t sW = base_s + stage * a.stage_bytes;
-        const uint32_t sN = sW + kBoxBytes;
-        if (kb < a.kb_main) {
-          tma_load_2d(sW, &tmW, &full[stage], kb * kBK, mt * kBM);
-          for (int b = 0; b < nboxes; ++b) tma_load_2d(sN + b * kBoxBytes, &tmA, &full[stage], kb * kBK, c0 + b * kBoxRows);
-        } else {
-          const int e = kb - a.kb_main;
-          tma_load_2d(sW, &tmB, &full[stage], e * kBK, mt * kBM);
-          for (int b = 0; b < nboxes; ++b) tma_load_2d(sN + b * kBoxBytes, &tmG, &full[stage], e * kBK, c0 + b * kBoxRows);
-        }
-        last_parity[stage] = phase;
-        if (filled < a.stages) ++filled;
-        if (++stage == a.stages) {
-          stage = 0;
-          phase ^= 1u;
+    // The whole warp runs the loop; lane 0 owns the ring bookkeeping and each
+    // lane issues at most one TMA box per stage (lane 0 the W-side box, lanes
+    // 1.. the N-side boxes), so the issue latency of one thread is not paid
+    // once per box.
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t parity_bits = 0;  // bit s: parity of the latest fill of stage s
+    uint32_t filled_mask = 0;
+    bool gram_ready = false;
+    bool ok = true;
+    auto acquire = [&](uint32_t bytes) -> bool {
+      bool got = true;
+      if (lane == 0) {
+        got = mbar_wait(&empty[stage], phase ^ 1u, limit);
+        if (got) mbar_arrive_expect_tx(&full[stage], bytes);
+        else record_timeout(a.status, abort_flag);
+      }
+      got = __shfl_sync(0xffffffffu, got, 0);
+      __syncwarp();
+      return got;
+    };
+    auto advance = [&]() {
+      parity_bits = (parity_bits & ~(1u << stage)) | (phase << stage);
+      filled_mask |= 1u << stage;
+      if (++stage == a.stages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    };
+    UnitIter x;
+    for (x.start(a, u_begin, u_end); x.valid() && ok; x.next(a)) {
+      const int nboxes = (x.n_this + kBoxRows - 1) / kBoxRows;
+      const bool ext = x.kb >= a.kb_main;
+      if (ext && !gram_ready) {
+        grid_dep_wait();  // G' is written by the Gram kernels
+        gram_ready = true;
+      }
+      if (!(ok = acquire(static_cast<uint32_t>(kBoxBytes * (1 + nboxes))))) break;
+      if (lane <= nboxes) {
+        const CUtensorMap* map = lane == 0 ? (ext ? &tmB : &tmW) : (ext ? &tmG : &tmA);
+        const int xk = (ext ? x.kb - a.kb_main : x.kb) * kBK;
+        const int y = lane == 0 ? x.mt * kBM : x.c0 + (lane - 1) * kBoxRows;
+        tma_load_2d(base_s + stage * a.stage_bytes + lane * kBoxBytes, map, &full[stage], xk, y);
+      }
+      advance();
+      if (x.seg_last(a)) {
+        // B[m tile rows, chunk columns] for the segment epilogue, 64 columns per box
+        const int nbox = (x.n_this + kBK - 1) / kBK;
+        for (int b0 = 0; b0 < nbox; b0 += slots) {
+          const int nb = min(slots, nbox - b0);
+          if (!(ok = acquire(static_cast<uint32_t>(kBoxBytes * nb)))) break;
+          if (lane < nb)
+            tma_load_2d(base_s + stage * a.stage_bytes + lane * kBoxBytes, &tmB, &full[stage],
+                        x.c0 + (b0 + lane) * kBK, x.mt * kBM);
+          advance();
         }
       }
-      // Never leave a TMA copy in flight: wait for the latest fill of every stage.
-      for (int s = 0; s < filled; ++s) mbar_wait(&full[s], last_parity[s], limit);
     }
+    // Never leave a TMA copy in flight: wait for the latest fill of every stage.
+    if (lane == 0)
+      for (int s2 = 0; s2 < a.stages; ++s2)
+        if ((filled_mask >> s2) & 1u) mbar_wait(&full[s2], (parity_bits >> s2) & 1u, limit);
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int seg = 0;
-      for (long long u = u_begin; u < u_end; ++u) {
-        if (*abort_flag) break;
-        const int tc = static_cast<int>(u / kb_total);
-        const int kb = static_cast<int>(u % kb_total);
-        const int ch = tc % a.n_chunks;
-        const int n_this = min(a.chunk_n, a.r - ch * a.chunk_n);
-        const bool seg_first = (u == u_begin) || kb == 0;
-        const bool seg_last = (u == u_end - 1) || kb == kb_total - 1;
-        if (seg_first && seg > 0) {
+      bool ok = true;
+      auto advance = [&]() {
+        if (++stage == a.stages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      };
+      auto fail = [&]() {
+        record_timeout(a.status, abort_flag);
+        ok = false;
+      };
+      UnitIter x;
+      int n_cur = -1;
+      uint32_t idesc0 = 0, idesc1 = 0;
+      for (x.start(a, u_begin, u_end); x.valid() && ok; x.next(a)) {
+        if (x.n_this != n_cur) {  // MMA pieces of N <= 256 for this chunk width
+          n_cur = x.n_this;
+          idesc0 = idesc_bf16_f32(kBM, min(256, n_cur));
+          idesc1 = n_cur > 256 ? idesc_bf16_f32(kBM, n_cur - 256) : 0u;
+        }
+        if (x.seg_first && seg > 0) {
           if (!mbar_wait(tmem_empty, static_cast<uint32_t>((seg - 1) & 1), limit)) {
-            record_timeout(a.status, abort_flag);
+            fail();
             break;
           }
           tc_fence_after();
         }
         if (!mbar_wait(&full[stage], phase, limit)) {
-          record_timeout(a.status, abort_flag);
+          fail();
           break;
         }
         tc_fence_after();
         const uint32_t sW = base_s + stage * a.stage_bytes;
-        const uint32_t sN = sW + kBoxBytes;
+        const uint64_t adesc = sw128_kmajor_desc(sW);
+        const uint64_t bdesc = sw128_kmajor_desc(sW + kBoxBytes);
 #pragma unroll
         for (int k = 0; k < kBK / 16; ++k) {
-          const uint64_t adesc = sw128_kmajor_desc(sW + k * 32);
-          for (int p = 0; p * 256 < n_this; ++p) {
-            const int pn = min(256, n_this - p * 256);
-            const uint64_t bdesc = sw128_kmajor_desc(sN + p * 256 * 128 + k * 32);
-            mma_bf16(tmem + p * 256, adesc, bdesc, idesc_bf16_f32(kBM, pn), (seg_first && k == 0) ? 0u : 1u);
-          }
+          // +32 bytes along K inside the swizzled row is +2 in the 16-byte address field
+          const uint32_t acc = (x.seg_first && k == 0) ? 0u : 1u;
+          mma_bf16(tmem, adesc + 2 * k, bdesc + 2 * k, idesc0, acc);
+          if (idesc1) mma_bf16(tmem + 256, adesc + 2 * k, bdesc + (256 * 128 >> 4) + 2 * k, idesc1, acc);
         }
         mma_commit(&empty[stage]);
-        if (seg_last) {
+        advance();
+        if (x.seg_last(a)) {
           mma_commit(tmem_full);
           ++seg;
-        }
-        if (++stage == a.stages) {
-          stage = 0;
-          phase ^= 1u;
+          // the B stages feed the epilogue only: release them on arrival
+          const int nbst = b_stages(a, x.n_this);
+          for (int i = 0; i < nbst; ++i) {
+            if (!mbar_wait(&full[stage], phase, limit)) {
+              fail();
+              break;
+            }
+            mbar_arrive(&empty[stage]);
+            advance();
+          }
         }
       }
       mma_commit(drain);
@@ -242,39 +334,32 @@ __global__ void __launch_bounds__(kNormThreads, 1)
     uint32_t phase = 0;
     int seg = 0;
     float base_acc = 0.f;
-    for (long long u = u_begin; u < u_end; ++u) {
-      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-      const int tc = static_cast<int>(u / kb_total);
-      const int kb = static_cast<int>(u % kb_total);
-      const int mt = tc / a.n_chunks;
-      const int ch = tc % a.n_chunks;
-      const int c0 = ch * a.chunk_n;
-      const int n_this = min(a.chunk_n, a.r - c0);
-      const bool seg_last = (u == u_end - 1) || kb == kb_total - 1;
-      if (!mbar_wait_warp(&full[stage], phase, limit)) {
-        if (lane == 0) record_timeout(a.status, abort_flag);
-        break;
-      }
-      if (ch == 0 && kb < a.kb_main) {
-        // ||W_i||^2 from the swizzled W stage: the 128-byte row of row_local
-        // holds its 64 K values with 16-byte chunks permuted; the sum does
-        // not care about the order, and visiting chunk (j ^ row % 8) keeps the
-        // eight rows of a quarter-warp on distinct banks.
-        const uint8_t* rowp = smem + stage * a.stage_bytes + row_local * 128;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint4 v = *reinterpret_cast<const uint4*>(rowp + ((j ^ (row_local & 7)) << 4));
-          base_acc += sumsq_bf16x8(v);
-        }
-      }
-      fence_proxy_async_smem();
+    bool deps_ready = false;
+    auto release = [&]() {
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[stage]);
       if (++stage == a.stages) {
         stage = 0;
         phase ^= 1u;
       }
-      if (!seg_last) continue;
+    };
+    UnitIter x;
+    for (x.start(a, u_begin, u_end); x.valid(); x.next(a)) {
+      if (__any_sync(0xffffffffu, !mbar_wait(&full[stage], phase, limit))) {
+        if (lane == 0) record_timeout(a.status, abort_flag);
+        break;
+      }
+      if (x.ch == 0 && x.kb < a.kb_main) {
+        // ||W_i||^2 from the swizzled W stage; the sum ignores the chunk
+        // order, and visiting chunk (j ^ row % 8) keeps the eight rows of a
+        // quarter-warp on distinct banks.
+        const uint8_t* tile = smem + stage * a.stage_bytes;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          base_acc += sumsq_bf16x8(*reinterpret_cast<const uint4*>(tile + sw128_chunk(row_local, j)));
+      }
+      release();
+      if (!x.seg_last(a)) continue;
 
       // ---- segment epilogue: <B_i, V_i> over this chunk's columns
       if (!mbar_wait_warp(tmem_full, static_cast<uint32_t>(seg & 1), limit)) {
@@ -282,21 +367,35 @@ __global__ void __launch_bounds__(kNormThreads, 1)
         break;
       }
       tc_fence_after();
-      const int row = mt * kBM + row_local;
-      const bool row_ok = row < a.d_out;
-      const __nv_bfloat16* brow = a.B + static_cast<size_t>(row_ok ? row : 0) * a.r + c0;
       float dot = 0.f;
-      for (int j0 = 0; j0 < n_this; j0 += 32) {
-        float acc[32];
-        tmem_ld32(tmem_lane + j0, acc);
-        if (row_ok) {
-          const uint4* bp = reinterpret_cast<const uint4*>(brow + j0);
-          const int nv = min(4, (n_this - j0) >> 3);
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            if (v < nv) dot += dot_bf16x8(__ldg(bp + v), acc + 8 * v);
+      const int nbox = (x.n_this + kBK - 1) / kBK;
+      bool ok = true;
+      for (int b0 = 0; b0 < nbox; b0 += slots) {
+        if (!mbar_wait_warp(&full[stage], phase, limit)) {
+          if (lane == 0) record_timeout(a.status, abort_flag);
+          ok = false;
+          break;
         }
+        const uint8_t* sb = smem + stage * a.stage_bytes;
+        const int nb = min(slots, nbox - b0);
+        for (int b = 0; b < nb; ++b) {
+          const uint8_t* tile = sb + b * kBoxBytes;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int j0 = (b0 + b) * kBK + h * 32;
+            if (j0 >= x.n_this) break;
+            float acc[32];
+            tmem_ld32(tmem_lane + j0, acc);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              if (j0 + 8 * v < x.n_this)
+                dot += dot_bf16x8(*reinterpret_cast<const uint4*>(tile + sw128_chunk(row_local, h * 4 + v)),
+                                  acc + 8 * v);
+          }
+        }
+        release();
       }
+      if (!ok) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tmem_empty);
@@ -304,34 +403,38 @@ __global__ void __launch_bounds__(kNormThreads, 1)
 
       const float partial = base_acc + a.two_s * dot;
       base_acc = 0.f;
-      a.partials[static_cast<size_t>(blockIdx.x + tc) * kBM + row_local] = partial;
+      if (!deps_ready) {
+        grid_dep_wait();  // counters are zeroed by the Gram reduction kernel
+        deps_ready = true;
+      }
+      a.partials[static_cast<size_t>(blockIdx.x + x.tc) * kBM + row_local] = partial;
 
       // ---- the last of the M tile's segment-warps to arrive finishes the tile
       __threadfence();
       __syncwarp();
       int expected = 0;
       for (int c2 = 0; c2 < a.n_chunks; ++c2) {
-        const long long s0 = static_cast<long long>(mt * a.n_chunks + c2) * kb_total;
-        expected += stream_k_owner(s0 + kb_total - 1, U, G) - stream_k_owner(s0, U, G) + 1;
+        const long long s0 = static_cast<long long>(x.mt * a.n_chunks + c2) * a.kb_total;
+        expected += stream_k_owner(s0 + a.kb_total - 1, U, G) - stream_k_owner(s0, U, G) + 1;
       }
       int last = 0;
-      if (lane == 0) last = (atomicAdd(&a.counters[mt], 1) == 4 * expected - 1);
+      if (lane == 0) last = (atomicAdd(&a.counters[x.mt], 1) == 4 * expected - 1);
       last = __shfl_sync(0xffffffffu, last, 0);
       if (last) {
         __threadfence();
         for (int rr = lane; rr < kBM; rr += 32) {
           float total = 0.f;
           for (int c2 = 0; c2 < a.n_chunks; ++c2) {
-            const int tc2 = mt * a.n_chunks + c2;
-            const long long s0 = static_cast<long long>(tc2) * kb_total;
+            const int tc2 = x.mt * a.n_chunks + c2;
+            const long long s0 = static_cast<long long>(tc2) * a.kb_total;
             const int o0 = stream_k_owner(s0, U, G);
-            const int o1 = stream_k_owner(s0 + kb_total - 1, U, G);
+            const int o1 = stream_k_owner(s0 + a.kb_total - 1, U, G);
             for (int o = o0; o <= o1; ++o) total += ld_cg_f32(&a.partials[static_cast<size_t>(o + tc2) * kBM + rr]);
           }
-          const int row2 = mt * kBM + rr;
+          const int row2 = x.mt * kBM + rr;
           if (row2 < a.d_out) a.n_out[row2] = sqrtf(fmaxf(total, 0.f));
         }
-        if (lane == 0) a.counters[mt] = 0;
+        if (lane == 0) a.counters[x.mt] = 0;
       }
     }
   }
@@ -346,14 +449,9 @@ __global__ void __launch_bounds__(kNormThreads, 1)
 struct GramArgs {
   int r, kb_main, splits, n_tiles;
   long long wait_limit;
-  float* partial;  // [splits][tri tiles][128][128] fp32, upper-triangular tiles (mi <= ni) packed
+  float* partial;  // [splits][n_tiles^2][128][128] fp32
   int* status;
 };
-
-// Index of upper-triangular tile (mi <= ni) among nt x nt tiles, row-major.
-__host__ __device__ __forceinline__ int tri_index(int mi, int ni, int nt) {
-  return mi * nt - mi * (mi - 1) / 2 + (ni - mi);
-}
 
 constexpr int kGramStages = 4;
 constexpr uint32_t kGramStageBytes = 2 * kBoxBytes;
@@ -374,17 +472,12 @@ __global__ void __launch_bounds__(kNormThreads, 1)
   const int lane = threadIdx.x & 31;
   const long long limit = a.wait_limit;
 
-  // (upper-triangular tile, K split) of this CTA
+  // (tile, K split) of this CTA; every tile of the n_tiles x n_tiles grid is
+  // computed so the reduction reads each output element contiguously
   const int split = blockIdx.x % a.splits;
   const int tile = blockIdx.x / a.splits;
-  const int n_tri = a.n_tiles * (a.n_tiles + 1) / 2;
-  int t = tile;
-  int mi = 0;
-  while (t >= a.n_tiles - mi) {
-    t -= a.n_tiles - mi;
-    ++mi;
-  }
-  const int ni = mi + t;
+  const int mi = tile / a.n_tiles;
+  const int ni = tile % a.n_tiles;
   const int n_this = min(kBoxRows, a.r - ni * kBoxRows);
   const int kb_lo = static_cast<int>(static_cast<long long>(split) * a.kb_main / a.splits);
   const int kb_hi = static_cast<int>(static_cast<long long>(split + 1) * a.kb_main / a.splits);
@@ -407,6 +500,7 @@ __global__ void __launch_bounds__(kNormThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dep_launch();  // the reduction kernel may be scheduled now; it waits for us
 
   if (warp == 0) {
     if (lane == 0) {
@@ -462,23 +556,20 @@ __global__ void __launch_bounds__(kNormThreads, 1)
   } else {
     const int q = warp & 3;
     const int row_local = q * 32 + lane;
-    const int row = mi * kBoxRows + row_local;
     const bool ok = mbar_wait_warp(tmem_full, 0, limit);
     if (ok && !__any_sync(0xffffffffu, *abort_flag != 0)) {
       tc_fence_after();
-      float* dst = a.partial + (static_cast<size_t>(split) * n_tri + tile) * (kBoxRows * kBoxRows) +
+      float* dst = a.partial + (static_cast<size_t>(split) * a.n_tiles * a.n_tiles + tile) * (kBoxRows * kBoxRows) +
                    static_cast<size_t>(row_local) * kBoxRows;
       for (int j0 = 0; j0 < n_this; j0 += 32) {
         float acc[32];
         tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + j0, acc);
-        if (row < a.r) {
-          const int nv = min(8, (n_this - j0) >> 2);
+        const int nv = min(8, (n_this - j0) >> 2);
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            if (v < nv)
-              reinterpret_cast<float4*>(dst + j0)[v] =
-                  make_float4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
-        }
+        for (int v = 0; v < 8; ++v)
+          if (v < nv)
+            reinterpret_cast<float4*>(dst + j0)[v] =
+                make_float4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
       }
     } else if (!ok && lane == 0) {
       record_timeout(a.status, abort_flag);
@@ -496,19 +587,19 @@ __global__ void __launch_bounds__(kNormThreads, 1)
 // tile counters.
 __global__ void gram_reduce_kernel(const float* __restrict__ partial, int splits, int r, float half_s,
                                    __nv_bfloat16* __restrict__ Gs, int* counters, int n_counters) {
+  grid_dep_launch();
+  grid_dep_wait();  // the Gram partial tiles are complete
   const long long total = static_cast<long long>(r) * r;
   const int nt = (r + kBoxRows - 1) / kBoxRows;
-  const long long split_stride = static_cast<long long>(nt * (nt + 1) / 2) * kBoxRows * kBoxRows;
+  const long long split_stride = static_cast<long long>(nt) * nt * kBoxRows * kBoxRows;
   for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
        idx += static_cast<long long>(gridDim.x) * blockDim.x) {
     const int j = static_cast<int>(idx / r);
     const int k = static_cast<int>(idx % r);
-    const bool upper = (j / kBoxRows) <= (k / kBoxRows);
-    const int rr = upper ? j : k, cc = upper ? k : j;  // element of the stored upper tile
-    const long long src = static_cast<long long>(tri_index(rr / kBoxRows, cc / kBoxRows, nt)) * kBoxRows * kBoxRows +
-                          static_cast<long long>(rr % kBoxRows) * kBoxRows + (cc % kBoxRows);
+    const long long src = (static_cast<long long>(j / kBoxRows) * nt + k / kBoxRows) * kBoxRows * kBoxRows +
+                          static_cast<long long>(j % kBoxRows) * kBoxRows + (k % kBoxRows);
     float sum = 0.f;
-    for (int s = 0; s < splits; ++s) sum += partial[s * split_stride + src];
+    for (int s = 0; s < splits; ++s) sum += __ldg(partial + s * split_stride + src);
     Gs[idx] = __float2bfloat16_rn(half_s * sum);
   }
   const int tid = blockIdx.x * blockDim.x + threadIdx.x;
