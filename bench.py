@@ -38,7 +38,8 @@ from factored_weight_norm_b200 import workloads as WL  # noqa: E402
 METRIC = "factored-norm TFLOP/s + fused-compose HBM GB/s (d=8192, r=384, bf16), % roofline"
 # bounded oracle sample per step: norm rows, compose tokens (about 1 s of CPU work)
 ORACLE_SAMPLE = (1024, 512)
-ORACLE_REPS = 10
+ORACLE_MIN_SECONDS = 10.0  # repeat the sample until this much CPU time is measured
+ORACLE_MAX_REPS = 200
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -108,7 +109,7 @@ class ClockSampler:
         self.path = f"/tmp/dora_clocks_{os.getpid()}.csv"
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "100"],
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
@@ -337,7 +338,7 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WL.HEADLINE.name, choices=sorted(WL.WORKLOADS))
@@ -394,10 +395,12 @@ def main():
 
     cpu = None
     if rank == 0 and N == 1 and not args.no_cpu_baseline:
-        obs = [time_oracle(wl, *ORACLE_SAMPLE) for _ in range(ORACLE_REPS)]
+        obs = []
+        while len(obs) < ORACLE_MAX_REPS and sum(o["t"] for o in obs) < ORACLE_MIN_SECONDS:
+            obs.append(time_oracle(wl, *ORACLE_SAMPLE, seed=len(obs)))
         cpu = {"value": statistics.median(o["norm_tflops"] for o in obs), "unit": "TFLOP/s",
                "cores": oracle_threads(), "kind": "oracle",
-               "sample": f"{obs[0]['sample']}; median of {ORACLE_REPS} repetitions",
+               "sample": f"{obs[0]['sample']}; median of {len(obs)} repetitions",
                "cpu_seconds": sum(o["t"] for o in obs),
                "compose_fwd_gbs": statistics.median(o["fwd_gbs"] for o in obs),
                "compose_bwd_gbs": statistics.median(o["bwd_gbs"] for o in obs)}

@@ -345,8 +345,10 @@ int dora_compose_fwd(const void* base_out, const void* lora_out, const float* m,
     occ = ctas_per_sm(compose_fwd_kernel<float, 4>, threads);
   else
     occ = ctas_per_sm(compose_fwd_kernel<float, 1>, threads);
-  const long long slots = static_cast<long long>(dev->num_sms) * occ;
-  const long long gy = pick_chunks(gx, slots, std::min<long long>(tokens, 65535));
+  // Several short waves of small CTAs stream better than one wave of long
+  // ones here: about 8 CTAs per SM in total, whatever the residency.
+  (void)occ;
+  const long long gy = std::max<long long>(1, std::min<long long>({8LL * dev->num_sms / gx, tokens, 65535}));
   const long long rows = cdiv(tokens, gy);
   const long long gy2 = cdiv(tokens, rows);
   dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy2));
