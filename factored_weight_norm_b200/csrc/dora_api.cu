@@ -466,3 +466,106 @@ int dora_num_sms(void) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------
+// dora_compose_bwd_noalloc: the compose backward with library-owned scratch.
+// The scratch is one file-scope device array; host code must not pass the
+// array's name to a kernel (on the host it is only a stand-in symbol), so its
+// device address is looked up once per device with that device current.
+namespace dora {
+namespace {
+
+constexpr int kNoallocChunks = 16;     // row chunks of column partials
+constexpr size_t kNoallocCounterBytes = 8192;
+static_assert(DORA_NOALLOC_SCRATCH_BYTES == kNoallocCounterBytes + kNoallocChunks * 4ull * DORA_NOALLOC_MAX_D_OUT,
+              "scratch layout and the header's size disagree");
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[DORA_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+unsigned char* g_noalloc_ptr[kMaxDevices] = {};
+
+int noalloc_scratch(unsigned char** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DORA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return DORA_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = static_cast<unsigned char*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return DORA_OK;
+}
+
+}  // namespace
+}  // namespace dora
+
+extern "C" int dora_compose_bwd_noalloc(const void* dy, const void* base_out, const void* lora_out, const float* m,
+                                        const float* n, float s, int64_t tokens, int64_t d_out, dora_dtype dt,
+                                        void* d_base, void* d_lora, float* d_m, void* stream) {
+  if (dt != DORA_BF16 && dt != DORA_F32) return DORA_ERR_UNSUPPORTED;
+  if (tokens < 0 || d_out < 0) return DORA_ERR_INVALID_ARG;
+  if (d_out > DORA_NOALLOC_MAX_D_OUT) return DORA_ERR_UNSUPPORTED;
+  if (d_out == 0) return DORA_OK;
+  if (!m || !n || !d_m) return DORA_ERR_INVALID_ARG;
+  if (tokens > 0 && (!dy || !base_out || !lora_out || !d_base || !d_lora)) return DORA_ERR_INVALID_ARG;
+  int vec = 1;
+  if (dt == DORA_BF16) {
+    if (d_out % 8 != 0) return DORA_ERR_UNSUPPORTED;
+    if (tokens > 0 && (!aligned(dy, 16) || !aligned(base_out, 16) || !aligned(lora_out, 16) ||
+                       !aligned(d_base, 16) || !aligned(d_lora, 16)))
+      return DORA_ERR_UNSUPPORTED;
+    vec = 8;
+  } else {
+    const bool a16 = aligned(dy, 16) && aligned(base_out, 16) && aligned(lora_out, 16) && aligned(d_base, 16) &&
+                     aligned(d_lora, 16);
+    if (!aligned(dy, 4) || !aligned(base_out, 4) || !aligned(lora_out, 4) || !aligned(d_base, 4) ||
+        !aligned(d_lora, 4))
+      return DORA_ERR_UNSUPPORTED;
+    vec = (d_out % 4 == 0 && a16) ? 4 : 1;
+  }
+  if (!aligned(m, 4) || !aligned(n, 4) || !aligned(d_m, 4)) return DORA_ERR_UNSUPPORTED;
+  DeviceInfo* dev = nullptr;
+  if (device_info(&dev)) return DORA_ERR_CUDA;
+  unsigned char* scratch = nullptr;
+  if (noalloc_scratch(&scratch)) return DORA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (tokens == 0) return cudaMemsetAsync(d_m, 0, static_cast<size_t>(d_out) * 4, st) == cudaSuccess ? DORA_OK : DORA_ERR_CUDA;
+
+  const long long nvec = d_out / vec;
+  const long long strips = cdiv(nvec, kBwdVecs);
+  int occ = 1;
+  if (dt == DORA_BF16)
+    occ = ctas_per_sm(compose_bwd_kernel<__nv_bfloat16, 8>, kBwdThreads);
+  else if (vec == 4)
+    occ = ctas_per_sm(compose_bwd_kernel<float, 4>, kBwdThreads);
+  else
+    occ = ctas_per_sm(compose_bwd_kernel<float, 1>, kBwdThreads);
+  const long long chunks = pick_chunks(strips, static_cast<long long>(dev->num_sms) * occ,
+                                       std::min<long long>(kNoallocChunks, cdiv(tokens, kBwdSlots)));
+  const long long rows = cdiv(tokens, chunks);
+  const long long chunks2 = cdiv(tokens, rows);
+  int* cnt = reinterpret_cast<int*>(scratch);
+  float* part = reinterpret_cast<float*>(scratch + kNoallocCounterBytes);
+  // the strip counters must start at zero; the partials are written before read
+  if (cudaMemsetAsync(cnt, 0, static_cast<size_t>(strips) * 4, st) != cudaSuccess) return DORA_ERR_CUDA;
+  dim3 grid(static_cast<unsigned>(strips), static_cast<unsigned>(chunks2));
+  if (dt == DORA_BF16)
+    compose_bwd_kernel<__nv_bfloat16, 8><<<grid, kBwdThreads, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(dy), static_cast<const __nv_bfloat16*>(base_out),
+        static_cast<const __nv_bfloat16*>(lora_out), m, n, s, tokens, nvec, d_out,
+        static_cast<__nv_bfloat16*>(d_base), static_cast<__nv_bfloat16*>(d_lora), part, cnt, d_m, rows);
+  else if (vec == 4)
+    compose_bwd_kernel<float, 4><<<grid, kBwdThreads, 0, st>>>(
+        static_cast<const float*>(dy), static_cast<const float*>(base_out), static_cast<const float*>(lora_out), m, n,
+        s, tokens, nvec, d_out, static_cast<float*>(d_base), static_cast<float*>(d_lora), part, cnt, d_m, rows);
+  else
+    compose_bwd_kernel<float, 1><<<grid, kBwdThreads, 0, st>>>(
+        static_cast<const float*>(dy), static_cast<const float*>(base_out), static_cast<const float*>(lora_out), m, n,
+        s, tokens, nvec, d_out, static_cast<float*>(d_base), static_cast<float*>(d_lora), part, cnt, d_m, rows);
+  return launch_error();
+}

@@ -45,6 +45,11 @@ SIGNATURES = {
         [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _f32, _i64, _i64, ctypes.c_int,
          _c_void_p, _c_void_p, _c_void_p, _c_void_p, _size, _c_void_p],
     ),
+    "dora_compose_bwd_noalloc": (
+        ctypes.c_int,
+        [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _f32, _i64, _i64, ctypes.c_int,
+         _c_void_p, _c_void_p, _c_void_p, _c_void_p],
+    ),
     "dora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "dora_device_status": (ctypes.c_int, [_c_void_p]),
     "dora_num_sms": (ctypes.c_int, []),

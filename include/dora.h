@@ -104,6 +104,36 @@ DORA_API int dora_compose_bwd(const void* dy, const void* base_out, const void* 
                      float s, int64_t tokens, int64_t d_out, dora_dtype dt, void* d_base, void* d_lora, float* d_m,
                      void* workspace, size_t workspace_bytes, void* stream);
 
+/* Largest d_out dora_compose_bwd_noalloc accepts, and the size of the
+ * library-owned scratch array behind it (8 KiB of counters + 16 row chunks of
+ * fp32 column partials). */
+#define DORA_NOALLOC_MAX_D_OUT 32768
+#define DORA_NOALLOC_SCRATCH_BYTES (8192 + 16 * 4 * DORA_NOALLOC_MAX_D_OUT)
+
+/* dora_compose_bwd for callers that cannot allocate device memory at call
+ * time and so cannot provide a workspace: code recorded into a CUDA graph or
+ * run under a runtime whose memory is fixed after initialisation, hot loops
+ * that must not call cudaMalloc/cudaFree, or foreign-language callers that
+ * only hold the tensors themselves.  This entry point has no counterpart on
+ * the pages; it computes exactly what dora_compose_bwd computes, with the
+ * same arguments minus the workspace.
+ *
+ * Its scratch lives in one file-scope device array of
+ * DORA_NOALLOC_SCRATCH_BYTES inside the library: every GPU that loads the
+ * library holds it until the process exits.  Nothing is allocated: no
+ * cudaMalloc, cudaFree or allocating library routine is called.  The first
+ * call on a device looks the array's device address up (cudaGetSymbolAddress)
+ * with that device current; make that first call before any stream capture.
+ * Each call clears the counters it needs (cudaMemsetAsync on the array) and
+ * the array otherwise keeps the last call's contents.  All calls on a device
+ * share the one array, so calls whose executions overlap on the GPU (for
+ * example on two streams without ordering between them) race and give wrong
+ * results; order them on one stream.  d_out > DORA_NOALLOC_MAX_D_OUT returns
+ * DORA_ERR_UNSUPPORTED and launches nothing. */
+DORA_API int dora_compose_bwd_noalloc(const void* dy, const void* base_out, const void* lora_out, const float* m,
+                                      const float* n, float s, int64_t tokens, int64_t d_out, dora_dtype dt,
+                                      void* d_base, void* d_lora, float* d_m, void* stream);
+
 /* Human-readable name of a dora_status value (static storage). */
 DORA_API const char* dora_status_string(int status);
 
