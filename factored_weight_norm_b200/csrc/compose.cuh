@@ -124,9 +124,10 @@ __global__ void __launch_bounds__(256, 3) compose_fwd_kernel(const T* __restrict
 constexpr int kBwdThreads = 256;  // 8 warps; a half-warp spans 16 vectors of one row
 constexpr int kBwdVecs = 16;      // vectors (column groups) per CTA strip
 constexpr int kBwdSlots = 16;     // rows visited concurrently by one CTA
+constexpr int kBwdRows = 4;       // rows in flight per thread
 
 template <typename T, int VEC>
-__global__ void __launch_bounds__(kBwdThreads, 3) compose_bwd_kernel(
+__global__ void __launch_bounds__(kBwdThreads, 2) compose_bwd_kernel(
     const T* __restrict__ dy, const T* __restrict__ base, const T* __restrict__ lora, const float* __restrict__ m,
     const float* __restrict__ n, float s, long long tokens, long long nvec, long long d_out, T* __restrict__ d_base,
     T* __restrict__ d_lora, float* __restrict__ partial, int* __restrict__ counters, float* __restrict__ d_m,
@@ -156,32 +157,30 @@ __global__ void __launch_bounds__(kBwdThreads, 3) compose_bwd_kernel(
     const long long row0 = blockIdx.y * rows_per_chunk;
     const long long row1 = min(tokens, row0 + rows_per_chunk);
     long long row = row0 + slot;
-    for (; row + kBwdSlots < row1; row += 2 * kBwdSlots) {
-      float a0[VEC], b0[VEC], l0[VEC], a1[VEC], b1[VEC], l1[VEC];
-      const long long o0 = row * d_out + col, o1 = (row + kBwdSlots) * d_out + col;
-      VecIO<T, VEC>::load(dy + o0, a0);
-      VecIO<T, VEC>::load(base + o0, b0);
-      VecIO<T, VEC>::load(lora + o0, l0);
-      VecIO<T, VEC>::load(dy + o1, a1);
-      VecIO<T, VEC>::load(base + o1, b1);
-      VecIO<T, VEC>::load(lora + o1, l1);
-      float db[VEC], dl[VEC];
+    // kBwdRows rows of this thread in flight: their three loads are issued
+    // before any is used
+    for (; row + (kBwdRows - 1) * kBwdSlots < row1; row += kBwdRows * kBwdSlots) {
+      float a[kBwdRows][VEC], b[kBwdRows][VEC], l[kBwdRows][VEC];
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) {
-        db[e] = g[e] * a0[e];
-        dl[e] = gs[e] * a0[e];
-        acc[e] = fmaf(a0[e], fmaf(s, l0[e], b0[e]), acc[e]);
+      for (int u = 0; u < kBwdRows; ++u) {
+        const long long o = (row + u * kBwdSlots) * d_out + col;
+        VecIO<T, VEC>::load(dy + o, a[u]);
+        VecIO<T, VEC>::load(base + o, b[u]);
+        VecIO<T, VEC>::load(lora + o, l[u]);
       }
-      VecIO<T, VEC>::store(d_base + o0, db);
-      VecIO<T, VEC>::store(d_lora + o0, dl);
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) {
-        db[e] = g[e] * a1[e];
-        dl[e] = gs[e] * a1[e];
-        acc[e] = fmaf(a1[e], fmaf(s, l1[e], b1[e]), acc[e]);
+      for (int u = 0; u < kBwdRows; ++u) {
+        const long long o = (row + u * kBwdSlots) * d_out + col;
+        float db[VEC], dl[VEC];
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+          db[e] = g[e] * a[u][e];
+          dl[e] = gs[e] * a[u][e];
+          acc[e] = fmaf(a[u][e], fmaf(s, l[u][e], b[u][e]), acc[e]);
+        }
+        VecIO<T, VEC>::store(d_base + o, db);
+        VecIO<T, VEC>::store(d_lora + o, dl);
       }
-      VecIO<T, VEC>::store(d_base + o1, db);
-      VecIO<T, VEC>::store(d_lora + o1, dl);
     }
     for (; row < row1; row += kBwdSlots) {
       float a0[VEC], b0[VEC], l0[VEC], db[VEC], dl[VEC];

@@ -203,7 +203,7 @@ int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_
   cfg.numAttrs = 1;
 
   const long long rr = static_cast<long long>(r) * r;
-  cfg.gridDim = dim3(static_cast<unsigned>(std::max<long long>(cdiv(p.m_tiles, 256), std::min<long long>(cdiv(rr, 256), 4 * dev->num_sms))));
+  cfg.gridDim = dim3(static_cast<unsigned>(std::max<long long>(cdiv(p.m_tiles, 256), std::min<long long>(cdiv(rr, 1024), 4 * dev->num_sms))));
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = 0;
   if (cudaLaunchKernelEx(&cfg, gram_reduce_kernel, static_cast<const float*>(Gp), ga.splits, static_cast<int>(r),
@@ -415,8 +415,9 @@ int dora_compose_bwd(const void* dy, const void* base_out, const void* lora_out,
     occ = ctas_per_sm(compose_bwd_kernel<float, 4>, kBwdThreads);
   else
     occ = ctas_per_sm(compose_bwd_kernel<float, 1>, kBwdThreads);
-  const long long chunks = pick_chunks(strips, static_cast<long long>(dev->num_sms) * occ,
-                                       std::min<long long>(kMaxBwdChunks, cdiv(tokens, kBwdSlots)));
+  // about two waves of resident CTAs
+  const long long chunks = std::max<long long>(
+      1, std::min<long long>({2LL * dev->num_sms * occ / strips, kMaxBwdChunks, cdiv(tokens, kBwdSlots)}));
   const long long rows = cdiv(tokens, chunks);
   const long long chunks2 = cdiv(tokens, rows);
   uint8_t* w = static_cast<uint8_t*>(workspace);

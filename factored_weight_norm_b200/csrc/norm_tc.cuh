@@ -453,8 +453,9 @@ struct GramArgs {
   int* status;
 };
 
-constexpr int kGramStages = 4;
-constexpr uint32_t kGramStageBytes = 2 * kBoxBytes;
+constexpr int kGramKPerStage = 2;  // K blocks per ring stage: 4 boxes, one per producer lane
+constexpr int kGramStages = 3;
+constexpr uint32_t kGramStageBytes = 2 * kGramKPerStage * kBoxBytes;
 
 __global__ void __launch_bounds__(kNormThreads, 1)
     gram_tc_kernel(const __grid_constant__ CUtensorMap tmA, const GramArgs a) {
@@ -503,47 +504,51 @@ __global__ void __launch_bounds__(kNormThreads, 1)
   grid_dep_launch();  // the reduction kernel may be scheduled now; it waits for us
 
   if (warp == 0) {
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t last_parity[kGramStages];
-      int filled = 0;
-      for (int kb = kb_lo; kb < kb_hi; ++kb) {
-        if (*abort_flag) break;
-        if (!mbar_wait(&empty[stage], phase ^ 1u, limit)) {
-          record_timeout(a.status, abort_flag);
-          break;
-        }
-        mbar_arrive_expect_tx(&full[stage], 2 * kBoxBytes);
-        const uint32_t sM = base_s + stage * kGramStageBytes;
-        tma_load_2d(sM, &tmA, &full[stage], kb * kBK, mi * kBoxRows);
-        tma_load_2d(sM + kBoxBytes, &tmA, &full[stage], kb * kBK, ni * kBoxRows);
-        last_parity[stage] = phase;
-        if (filled < kGramStages) ++filled;
-        if (++stage == kGramStages) {
-          stage = 0;
-          phase ^= 1u;
-        }
+    // lane 2i loads the M-side rows, lane 2i+1 the N-side rows, of K block kb0 + i
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t parity_bits = 0, filled_mask = 0;
+    for (int kb0 = kb_lo; kb0 < kb_hi; kb0 += kGramKPerStage) {
+      const int nk = min(kGramKPerStage, kb_hi - kb0);
+      bool got = true;
+      if (lane == 0) {
+        got = mbar_wait(&empty[stage], phase ^ 1u, limit);
+        if (got) mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(2 * nk * kBoxBytes));
+        else record_timeout(a.status, abort_flag);
       }
-      for (int s = 0; s < filled; ++s) mbar_wait(&full[s], last_parity[s], limit);
+      if (!__shfl_sync(0xffffffffu, got, 0)) break;
+      __syncwarp();
+      if (lane < 2 * nk)
+        tma_load_2d(base_s + stage * kGramStageBytes + lane * kBoxBytes, &tmA, &full[stage], (kb0 + (lane >> 1)) * kBK,
+                    ((lane & 1) ? ni : mi) * kBoxRows);
+      parity_bits = (parity_bits & ~(1u << stage)) | (phase << stage);
+      filled_mask |= 1u << stage;
+      if (++stage == kGramStages) {
+        stage = 0;
+        phase ^= 1u;
+      }
     }
+    if (lane == 0)
+      for (int s2 = 0; s2 < kGramStages; ++s2)
+        if ((filled_mask >> s2) & 1u) mbar_wait(&full[s2], (parity_bits >> s2) & 1u, limit);
   } else if (warp == 1) {
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      for (int kb = kb_lo; kb < kb_hi; ++kb) {
-        if (*abort_flag) break;
+      const uint32_t idesc = idesc_bf16_f32(kBM, n_this);
+      for (int kb0 = kb_lo; kb0 < kb_hi; kb0 += kGramKPerStage) {
+        const int nk = min(kGramKPerStage, kb_hi - kb0);
         if (!mbar_wait(&full[stage], phase, limit)) {
           record_timeout(a.status, abort_flag);
           break;
         }
         tc_fence_after();
-        const uint32_t sM = base_s + stage * kGramStageBytes;
+        const uint64_t d0 = sw128_kmajor_desc(base_s + stage * kGramStageBytes);
+        for (int i = 0; i < nk; ++i)
 #pragma unroll
-        for (int k = 0; k < kBK / 16; ++k) {
-          mma_bf16(tmem, sw128_kmajor_desc(sM + k * 32), sw128_kmajor_desc(sM + kBoxBytes + k * 32),
-                   idesc_bf16_f32(kBM, n_this), (kb == kb_lo && k == 0) ? 0u : 1u);
-        }
+          for (int k = 0; k < kBK / 16; ++k)
+            mma_bf16(tmem, d0 + (2 * i) * (kBoxBytes >> 4) + 2 * k, d0 + (2 * i + 1) * (kBoxBytes >> 4) + 2 * k, idesc,
+                     (kb0 == kb_lo && i == 0 && k == 0) ? 0u : 1u);
         mma_commit(&empty[stage]);
         if (++stage == kGramStages) {
           stage = 0;
@@ -592,15 +597,37 @@ __global__ void gram_reduce_kernel(const float* __restrict__ partial, int splits
   const long long total = static_cast<long long>(r) * r;
   const int nt = (r + kBoxRows - 1) / kBoxRows;
   const long long split_stride = static_cast<long long>(nt) * nt * kBoxRows * kBoxRows;
-  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
-       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int j = static_cast<int>(idx / r);
-    const int k = static_cast<int>(idx % r);
-    const long long src = (static_cast<long long>(j / kBoxRows) * nt + k / kBoxRows) * kBoxRows * kBoxRows +
-                          static_cast<long long>(j % kBoxRows) * kBoxRows + (k % kBoxRows);
-    float sum = 0.f;
-    for (int s = 0; s < splits; ++s) sum += __ldg(partial + s * split_stride + src);
-    Gs[idx] = __float2bfloat16_rn(half_s * sum);
+  // four elements per thread and eight splits per round: 32 independent loads
+  // in flight; each element still adds its splits in increasing order
+  constexpr int kE = 4, kS = 8;
+  const long long step = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long base = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; base < total;
+       base += kE * step) {
+    long long src[kE];
+    float sum[kE];
+#pragma unroll
+    for (int e = 0; e < kE; ++e) {
+      const long long idx = min(base + e * step, total - 1);
+      const int j = static_cast<int>(idx / r);
+      const int k = static_cast<int>(idx - static_cast<long long>(j) * r);
+      src[e] = (static_cast<long long>(j / kBoxRows) * nt + k / kBoxRows) * kBoxRows * kBoxRows +
+               static_cast<long long>(j % kBoxRows) * kBoxRows + (k % kBoxRows);
+      sum[e] = 0.f;
+    }
+    for (int s0 = 0; s0 < splits; s0 += kS) {
+      float v[kE][kS];
+#pragma unroll
+      for (int e = 0; e < kE; ++e)
+#pragma unroll
+        for (int t = 0; t < kS; ++t) v[e][t] = (s0 + t < splits) ? __ldg(partial + (s0 + t) * split_stride + src[e]) : 0.f;
+#pragma unroll
+      for (int e = 0; e < kE; ++e)
+#pragma unroll
+        for (int t = 0; t < kS; ++t) sum[e] += v[e][t];
+    }
+#pragma unroll
+    for (int e = 0; e < kE; ++e)
+      if (base + e * step < total) Gs[base + e * step] = __float2bfloat16_rn(half_s * sum[e]);
   }
   const int tid = blockIdx.x * blockDim.x + threadIdx.x;
   if (tid < n_counters) counters[tid] = 0;
