@@ -40,6 +40,7 @@ constexpr int kNormThreads = 192;     // warp 0 TMA, warp 1 MMA, warps 2..5 epil
 constexpr int kMaxChunkN = 512;       // TMEM columns
 constexpr int kMaxStages = 8;
 constexpr int kStatusTimeout = 5;     // == DORA_ERR_TIMEOUT
+constexpr int kFinOwners = 4;         // partial owners the finalizing warp loads together
 
 struct NormArgs {
   int d_out, d_in, r;
@@ -422,17 +423,37 @@ __global__ void __launch_bounds__(kNormThreads, 1)
       last = __shfl_sync(0xffffffffu, last, 0);
       if (last) {
         __threadfence();
-        for (int rr = lane; rr < kBM; rr += 32) {
-          float total = 0.f;
-          for (int c2 = 0; c2 < a.n_chunks; ++c2) {
-            const int tc2 = x.mt * a.n_chunks + c2;
-            const long long s0 = static_cast<long long>(tc2) * a.kb_total;
-            const int o0 = stream_k_owner(s0, U, G);
-            const int o1 = stream_k_owner(s0 + a.kb_total - 1, U, G);
-            for (int o = o0; o <= o1; ++o) total += ld_cg_f32(&a.partials[static_cast<size_t>(o + tc2) * kBM + rr]);
+        // lane l owns rows l, l + 32, l + 64, l + 96; the partials of up to
+        // kFinOwners owners are loaded together, then added in owner order
+        constexpr int kRows = kBM / 32;
+        float total[kRows];
+#pragma unroll
+        for (int j = 0; j < kRows; ++j) total[j] = 0.f;
+        for (int c2 = 0; c2 < a.n_chunks; ++c2) {
+          const int tc2 = x.mt * a.n_chunks + c2;
+          const long long s0 = static_cast<long long>(tc2) * a.kb_total;
+          const int o0 = stream_k_owner(s0, U, G);
+          const int o1 = stream_k_owner(s0 + a.kb_total - 1, U, G);
+          for (int ob = o0; ob <= o1; ob += kFinOwners) {
+            float v[kFinOwners][kRows];
+#pragma unroll
+            for (int k = 0; k < kFinOwners; ++k)
+#pragma unroll
+              for (int j = 0; j < kRows; ++j)
+                v[k][j] = (ob + k <= o1)
+                              ? ld_cg_f32(&a.partials[static_cast<size_t>(ob + k + tc2) * kBM + lane + 32 * j])
+                              : 0.f;
+#pragma unroll
+            for (int k = 0; k < kFinOwners; ++k)
+#pragma unroll
+              for (int j = 0; j < kRows; ++j)
+                if (ob + k <= o1) total[j] += v[k][j];
           }
-          const int row2 = x.mt * kBM + rr;
-          if (row2 < a.d_out) a.n_out[row2] = sqrtf(fmaxf(total, 0.f));
+        }
+#pragma unroll
+        for (int j = 0; j < kRows; ++j) {
+          const int row2 = x.mt * kBM + lane + 32 * j;
+          if (row2 < a.d_out) a.n_out[row2] = sqrtf(fmaxf(total[j], 0.f));
         }
         if (lane == 0) a.counters[x.mt] = 0;
       }
