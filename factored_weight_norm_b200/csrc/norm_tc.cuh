@@ -229,6 +229,12 @@ __global__ void __launch_bounds__(kNormThreads, 1)
     for (x.start(a, u_begin, u_end); x.valid() && ok; x.next(a)) {
       const int nboxes = (x.n_this + kBoxRows - 1) / kBoxRows;
       const bool ext = x.kb >= a.kb_main;
+      if (x.seg_first) {
+        // B's rows for this segment's epilogue: into L2 now, so that the ring
+        // loads of them at the segment end do not wait for HBM
+        const int nbox = (x.n_this + kBK - 1) / kBK;
+        for (int b = lane; b < nbox; b += 32) tma_prefetch_l2_2d(&tmB, x.c0 + b * kBK, x.mt * kBM);
+      }
       if (ext && !gram_ready) {
         grid_dep_wait();  // G' is written by the Gram kernels
         gram_ready = true;
