@@ -338,16 +338,8 @@ int dora_compose_fwd(const void* base_out, const void* lora_out, const float* m,
   const int threads = static_cast<int>(std::min<long long>(256, align_up(static_cast<size_t>(nvec), 32)));
   const long long gx = cdiv(nvec, threads);
   if (gx > INT32_MAX) return DORA_ERR_UNSUPPORTED;
-  int occ = 1;
-  if (dt == DORA_BF16)
-    occ = ctas_per_sm(compose_fwd_kernel<__nv_bfloat16, 8>, threads);
-  else if (vec == 4)
-    occ = ctas_per_sm(compose_fwd_kernel<float, 4>, threads);
-  else
-    occ = ctas_per_sm(compose_fwd_kernel<float, 1>, threads);
   // Several short waves of small CTAs stream better than one wave of long
   // ones here: about 8 CTAs per SM in total, whatever the residency.
-  (void)occ;
   const long long gy = std::max<long long>(1, std::min<long long>({8LL * dev->num_sms / gx, tokens, 65535}));
   const long long rows = cdiv(tokens, gy);
   const long long gy2 = cdiv(tokens, rows);
