@@ -142,6 +142,15 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------- our arm
+def max_over_ranks(values, world, device):
+    """Element-wise maximum of a list of floats over all ranks (the slowest
+    rank's time decides every multi-GPU number); identity when world == 1."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
 def run_ours(args, rank, world, local_rank):
     from factored_weight_norm_b200 import dora as D
 
@@ -199,10 +208,7 @@ def run_ours(args, rank, world, local_rank):
     t_fwd = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps * 1e-3
     t_bwd = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps * 1e-3
     t_total = evs[0][0].elapsed_time(evs[-1][3]) * 1e-3
-    times = torch.tensor([t_total, t_norm, t_fwd, t_bwd], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
-    t_total, t_norm, t_fwd, t_bwd = times.tolist()
+    t_total, t_norm, t_fwd, t_bwd = max_over_ranks([t_total, t_norm, t_fwd, t_bwd], world, dev)
 
     # ---- end to end through the Python API with pinned host buffers
     e2e = run_e2e(args, D, dev, wl, W, A, B, m, base, lora, dy, n, y, d_base, d_lora, d_m, ws_n, ws_b, world)
@@ -252,12 +258,9 @@ def run_e2e(args, D, dev, wl, W, A, B, m, base, lora, dy, n, y, d_base, d_lora, 
     for i in range(k):
         step(evs[i])
     torch.cuda.synchronize()
-    t = torch.tensor([sum(e[0].elapsed_time(e[1]) for e in evs) / k * 1e-3,
-                      sum(e[1].elapsed_time(e[2]) for e in evs) / k * 1e-3,
-                      sum(e[2].elapsed_time(e[3]) for e in evs) / k * 1e-3], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    t_norm, t_fwd, t_bwd = t.tolist()
+    t_norm, t_fwd, t_bwd = max_over_ranks([sum(e[0].elapsed_time(e[1]) for e in evs) / k * 1e-3,
+                                           sum(e[1].elapsed_time(e[2]) for e in evs) / k * 1e-3,
+                                           sum(e[2].elapsed_time(e[3]) for e in evs) / k * 1e-3], world, dev)
     return dict(t_norm=t_norm, t_fwd=t_fwd, t_bwd=t_bwd, h2d=h2d, d2h=d2h, steps=k)
 
 
@@ -334,6 +337,85 @@ def run_reference(args, rank, world):
     return 0
 
 
+def build_line(args, res, N, peaks, peak_src, traffic, cpu):
+    """The JSON line of our arm from the max-over-ranks times in `res`; N ranks
+    each ran one replica of the workload, so every rate is the whole job's."""
+    wl = res["wl"]
+    F = norm_flops(wl.d_out, wl.d_in, wl.r)
+    Bn = norm_bytes(wl.d_out, wl.d_in, wl.r)
+    Bf = fwd_bytes(wl.tokens, wl.d_out)
+    Bb = bwd_bytes(wl.tokens, wl.d_out)
+
+    def roof(kernel, t, work, bound):
+        if bound == "tensor":
+            ach = work / t / 1e12
+            pk = peaks["bf16_tflops"]
+            unit = "TFLOP/s"
+        else:
+            ach = work / t / 1e9
+            pk = peaks["hbm_gbs"]
+            unit = "GB/s"
+        tr = traffic.get(kernel)
+        return {"kernel": kernel, "bound": bound, "achieved": ach, "peak": pk, "unit": unit, "frac": ach / pk,
+                "traffic": tr["bytes"] if tr else None, "peak_source": f"{peak_src} (burst)" if bound == "tensor" else peak_src,
+                "time_us": t * 1e6}
+
+    # norm bound: slower of FLOPs at tensor peak and bytes at HBM bandwidth
+    norm_bound = "tensor" if F / (peaks["bf16_tflops"] * 1e12) >= Bn / (peaks["hbm_gbs"] * 1e9) else "hbm"
+    rl = [
+        roof("norm", res["t_norm"], F if norm_bound == "tensor" else Bn, norm_bound),
+        roof("compose_fwd", res["t_fwd"], Bf, "hbm"),
+        roof("compose_bwd", res["t_bwd"], Bb, "hbm"),
+    ]
+    dominant = max(rl, key=lambda x: x["time_us"])
+    e2e = res["e2e"]
+    e2e_norm = F * N / (e2e["t_norm"]) / 1e12
+
+    launches_per_step = 3 + 1 + 1  # gram, gram_reduce, norm; compose fwd; compose bwd
+    line = {
+        "metric": METRIC,
+        "value": F * N / res["t_norm"] / 1e12,
+        "unit": "TFLOP/s",
+        "n_gpus": N,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": res["t_total"] / args.steps * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "d_out": wl.d_out, "d_in": wl.d_in, "r": wl.r, "tokens": wl.tokens,
+                   "s": wl.s, "parallelism": f"replicas x{N}",
+                   "l2": "no flush: each step streams > 1 GB (W 134 MB, 3 activation reads + 3 writes of 134 MB)"},
+        "value_basis": "norm FLOPs x ranks / max-over-ranks mean CUDA-event time of the norm launches in the timed steps",
+        "compose": {
+            "fwd": {"value": Bf * N / res["t_fwd"] / 1e9, "unit": "GB/s", "frac": rl[1]["frac"],
+                    "time_us": res["t_fwd"] * 1e6},
+            "bwd": {"value": Bb * N / res["t_bwd"] / 1e9, "unit": "GB/s", "frac": rl[2]["frac"],
+                    "time_us": res["t_bwd"] * 1e6},
+        },
+        "norm": {"tflops": F / res["t_norm"] / 1e12, "frac": rl[0]["frac"], "bound": norm_bound,
+                 "time_us": res["t_norm"] * 1e6, "flops": F, "bytes": Bn},
+        "roofline": {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
+                    | {"kernel": dominant["kernel"], "peak_source": dominant["peak_source"]},
+        "rooflines": rl,
+        "step_roofline_frac": (
+            max(F / (peaks["bf16_tflops"] * 1e12), Bn / (peaks["hbm_gbs"] * 1e9))
+            + Bf / (peaks["hbm_gbs"] * 1e9) + Bb / (peaks["hbm_gbs"] * 1e9)) / (res["t_total"] / args.steps),
+        "e2e": {"value": e2e_norm, "unit": "TFLOP/s", "h2d_bytes_per_step": e2e["h2d"],
+                "d2h_bytes_per_step": e2e["d2h"], "steps": e2e["steps"],
+                "basis": "norm FLOPs / (H2D of W, A, B + norm + D2H of n), pinned host buffers",
+                "compose_fwd_gbs": Bf * N / e2e["t_fwd"] / 1e9, "compose_bwd_gbs": Bb * N / e2e["t_bwd"] / 1e9},
+        "cpu_baseline": cpu,
+        "gpu_launches": launches_per_step * args.steps,
+        "memset_nodes": args.steps,
+        "clocks": res["clocks"],
+        "device_status": res["status"],
+    }
+    return line
+
+
 # ------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -361,38 +443,8 @@ def main():
     res = run_ours(args, rank, world, local_rank)
     wl = res["wl"]
     N = world
-    F = norm_flops(wl.d_out, wl.d_in, wl.r)
-    Bn = norm_bytes(wl.d_out, wl.d_in, wl.r)
-    Bf = fwd_bytes(wl.tokens, wl.d_out)
-    Bb = bwd_bytes(wl.tokens, wl.d_out)
     peaks, peak_src = load_peaks()
     traffic = load_traffic()
-
-    def roof(kernel, t, work, bound):
-        if bound == "tensor":
-            ach = work / t / 1e12
-            pk = peaks["bf16_tflops"]
-            unit = "TFLOP/s"
-        else:
-            ach = work / t / 1e9
-            pk = peaks["hbm_gbs"]
-            unit = "GB/s"
-        tr = traffic.get(kernel)
-        return {"kernel": kernel, "bound": bound, "achieved": ach, "peak": pk, "unit": unit, "frac": ach / pk,
-                "traffic": tr["bytes"] if tr else None, "peak_source": f"{peak_src} (burst)" if bound == "tensor" else peak_src,
-                "time_us": t * 1e6}
-
-    # norm bound: slower of FLOPs at tensor peak and bytes at HBM bandwidth
-    norm_bound = "tensor" if F / (peaks["bf16_tflops"] * 1e12) >= Bn / (peaks["hbm_gbs"] * 1e9) else "hbm"
-    rl = [
-        roof("norm", res["t_norm"], F if norm_bound == "tensor" else Bn, norm_bound),
-        roof("compose_fwd", res["t_fwd"], Bf, "hbm"),
-        roof("compose_bwd", res["t_bwd"], Bb, "hbm"),
-    ]
-    dominant = max(rl, key=lambda x: x["time_us"])
-    e2e = res["e2e"]
-    e2e_norm = F * N / (e2e["t_norm"]) / 1e12
-
     cpu = None
     if rank == 0 and N == 1 and not args.no_cpu_baseline:
         obs = []
@@ -405,50 +457,8 @@ def main():
                "compose_fwd_gbs": statistics.median(o["fwd_gbs"] for o in obs),
                "compose_bwd_gbs": statistics.median(o["bwd_gbs"] for o in obs)}
 
-    launches_per_step = 3 + 1 + 1  # gram, gram_reduce, norm; compose fwd; compose bwd
     if rank == 0:
-        line = {
-            "metric": METRIC,
-            "value": F * N / res["t_norm"] / 1e12,
-            "unit": "TFLOP/s",
-            "n_gpus": N,
-            "steps": args.steps,
-            "warmup": args.warmup,
-            "ms_per_step": res["t_total"] / args.steps * 1e3,
-            "higher_is_better": True,
-            "scaling": "weak",
-            "vs_baseline": None,
-            "dtype": "bf16",
-            "data": "synthetic",
-            "config": {"workload": wl.name, "d_out": wl.d_out, "d_in": wl.d_in, "r": wl.r, "tokens": wl.tokens,
-                       "s": wl.s, "parallelism": f"replicas x{N}",
-                       "l2": "no flush: each step streams > 1 GB (W 134 MB, 3 activation reads + 3 writes of 134 MB)"},
-            "value_basis": "norm FLOPs x ranks / max-over-ranks mean CUDA-event time of the norm launches in the timed steps",
-            "compose": {
-                "fwd": {"value": Bf * N / res["t_fwd"] / 1e9, "unit": "GB/s", "frac": rl[1]["frac"],
-                        "time_us": res["t_fwd"] * 1e6},
-                "bwd": {"value": Bb * N / res["t_bwd"] / 1e9, "unit": "GB/s", "frac": rl[2]["frac"],
-                        "time_us": res["t_bwd"] * 1e6},
-            },
-            "norm": {"tflops": F / res["t_norm"] / 1e12, "frac": rl[0]["frac"], "bound": norm_bound,
-                     "time_us": res["t_norm"] * 1e6, "flops": F, "bytes": Bn},
-            "roofline": {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
-                        | {"kernel": dominant["kernel"], "peak_source": dominant["peak_source"]},
-            "rooflines": rl,
-            "step_roofline_frac": (
-                max(F / (peaks["bf16_tflops"] * 1e12), Bn / (peaks["hbm_gbs"] * 1e9))
-                + Bf / (peaks["hbm_gbs"] * 1e9) + Bb / (peaks["hbm_gbs"] * 1e9)) / (res["t_total"] / args.steps),
-            "e2e": {"value": e2e_norm, "unit": "TFLOP/s", "h2d_bytes_per_step": e2e["h2d"],
-                    "d2h_bytes_per_step": e2e["d2h"], "steps": e2e["steps"],
-                    "basis": "norm FLOPs / (H2D of W, A, B + norm + D2H of n), pinned host buffers",
-                    "compose_fwd_gbs": Bf * N / e2e["t_fwd"] / 1e9, "compose_bwd_gbs": Bb * N / e2e["t_bwd"] / 1e9},
-            "cpu_baseline": cpu,
-            "gpu_launches": launches_per_step * args.steps,
-            "memset_nodes": args.steps,
-            "clocks": res["clocks"],
-            "device_status": res["status"],
-        }
-        print(json.dumps(line), flush=True)
+        print(json.dumps(build_line(args, res, N, peaks, peak_src, traffic, cpu)), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
     return 0

@@ -1,0 +1,108 @@
+"""bench.py's multi-rank host logic on CPU: two gloo ranks (no GPU).
+
+One process per rank, as under torchrun.  Each rank reports different times;
+both must see the element-wise maximum (the slowest rank decides every number),
+rank 0 alone builds the JSON line, whose rates count the work of both replicas,
+and the reference arm runs on rank 0 only.
+"""
+
+import importlib.util
+import io
+import json
+import os
+import socket
+import contextlib
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        bench = _bench()
+        # rank k is slower on a different quantity than the other rank
+        mine = [1.0 + rank, 0.5 + 0.25 * (1 - rank), 0.1 + 0.05 * rank, 0.2]
+        got = bench.max_over_ranks(mine, world, torch.device("cpu"))
+        result = {"max": got}
+        if rank == 0:
+            wl = bench.WL.HEADLINE
+            res = dict(t_total=got[0], t_norm=got[1], t_fwd=got[2], t_bwd=got[3], clocks=None, status=0, wl=wl,
+                       e2e=dict(t_norm=2 * got[1], t_fwd=2 * got[2], t_bwd=2 * got[3], h2d=10, d2h=20, steps=5))
+
+            class Args:
+                steps, warmup = 7, 3
+
+            peaks = {"bf16_tflops": 1000.0, "hbm_gbs": 5000.0}
+            line = bench.build_line(Args, res, world, peaks, "test", {}, None)
+            result["line"] = json.loads(json.dumps(line))
+        # the reference arm: rank 0 only (rank 1 returns at once, printing nothing)
+        if rank == 1:
+            buf = io.StringIO()
+
+            class RefArgs:
+                steps, warmup, gpus, workload = 1, 0, world, bench.WL.HEADLINE.name
+
+            with contextlib.redirect_stdout(buf):
+                rc = bench.run_reference(RefArgs, rank, world)
+            result["ref_rc"] = rc
+            result["ref_out"] = buf.getvalue()
+        dist.barrier()
+        with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
+            json.dump(result, f)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.fixture(scope="module")
+def two_ranks(tmp_path_factory):
+    out = str(tmp_path_factory.mktemp("ranks"))
+    mp.start_processes(_rank_main, args=(2, _free_port(), out), nprocs=2, join=True, start_method="spawn")
+    return [json.load(open(os.path.join(out, f"rank{r}.json"))) for r in range(2)]
+
+
+def test_every_rank_sees_the_max(two_ranks):
+    expect = [2.0, 0.75, 0.15, 0.2]
+    for r in two_ranks:
+        assert r["max"] == pytest.approx(expect)
+
+
+def test_line_counts_both_replicas(two_ranks):
+    bench = _bench()
+    line = two_ranks[0]["line"]
+    wl = bench.WL.HEADLINE
+    F = bench.norm_flops(wl.d_out, wl.d_in, wl.r)
+    assert line["n_gpus"] == 2 and line["scaling"] == "weak"
+    assert line["config"]["parallelism"] == "replicas x2"
+    assert line["value"] == pytest.approx(2 * F / 0.75 / 1e12)
+    assert line["compose"]["fwd"]["value"] == pytest.approx(2 * bench.fwd_bytes(wl.tokens, wl.d_out) / 0.15 / 1e9)
+    assert line["compose"]["bwd"]["value"] == pytest.approx(2 * bench.bwd_bytes(wl.tokens, wl.d_out) / 0.2 / 1e9)
+    assert line["ms_per_step"] == pytest.approx(2.0 / 7 * 1e3)
+    # roofline fractions are per replica (one GPU's kernel against one GPU's peak)
+    assert line["norm"]["frac"] == pytest.approx(F / 0.75 / 1e12 / 1000.0)
+    assert line["roofline"]["kernel"] == "norm" and line["roofline"]["traffic"] is None
+    assert line["e2e"]["value"] == pytest.approx(2 * F / 1.5 / 1e12)
+
+
+def test_reference_arm_runs_on_rank_zero_only(two_ranks):
+    assert two_ranks[1]["ref_rc"] == 0
+    assert two_ranks[1]["ref_out"] == ""
+    assert "line" not in two_ranks[1]
