@@ -447,6 +447,14 @@ int dora_device_status(void* stream) {
   return v;
 }
 
+int dora_selftest_timeout(int64_t limit_cycles, void* stream) {
+  if (limit_cycles <= 0 || limit_cycles > kWaitLimitCycles) return DORA_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  if (device_info(&dev)) return DORA_ERR_CUDA;
+  timeout_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_cycles, dev->status);
+  return launch_error();
+}
+
 int dora_num_sms(void) {
   int n = 0;
   if (cudaGetDeviceCount(&n) != cudaSuccess || n == 0) {

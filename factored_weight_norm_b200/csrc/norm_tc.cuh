@@ -472,6 +472,23 @@ __global__ void __launch_bounds__(kNormThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, a.tmem_cols);
 }
 
+// ============================================================== self-test
+// One warp waits, bounded by `limit` cycles, on an mbarrier phase that nothing
+// completes, and takes the same exit as every other bounded wait here: the
+// timeout status is recorded and the kernel returns.  Exercises the failure
+// path (status word, host read-back, context still usable) without a fault.
+__global__ void timeout_probe_kernel(long long limit, int* status) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (!mbar_wait_warp(&bar, 0, limit) && threadIdx.x == 0) record_timeout(status, &abort_flag);
+}
+
 // ===================================================================== Gram
 struct GramArgs {
   int r, kb_main, splits, n_tiles;

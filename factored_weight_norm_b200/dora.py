@@ -53,6 +53,7 @@ SIGNATURES = {
     "dora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "dora_device_status": (ctypes.c_int, [_c_void_p]),
     "dora_num_sms": (ctypes.c_int, []),
+    "dora_selftest_timeout": (ctypes.c_int, [_i64, _c_void_p]),
 }
 
 _lib = None
@@ -133,6 +134,11 @@ def dora_num_sms() -> int:
 
 def dora_device_status(stream=None) -> int:
     return int(lib().dora_device_status(_stream(stream)))
+
+
+def dora_selftest_timeout(limit_cycles: int, stream=None) -> None:
+    """Runs the bounded-wait failure path once (see include/dora.h)."""
+    _check(lib().dora_selftest_timeout(int(limit_cycles), _stream(stream)), "dora_selftest_timeout")
 
 
 def dora_status_string(status: int) -> str:

@@ -141,6 +141,15 @@ DORA_API const char* dora_status_string(int status);
  * (DORA_OK or DORA_ERR_TIMEOUT).  Synchronises `stream` first. */
 DORA_API int dora_device_status(void* stream);
 
+/* Self-test of the failure path; no counterpart on the pages.  Launches one
+ * warp that waits on an mbarrier phase nothing completes, bounded by
+ * limit_cycles SM cycles (1 .. 2e9; about 1 s at 2 GHz), then records
+ * DORA_ERR_TIMEOUT in the device-side status word exactly as a real bounded
+ * wait that gives up does.  dora_device_status() then returns (and clears)
+ * DORA_ERR_TIMEOUT; the context stays usable.  Asynchronous on `stream`.
+ * Returns DORA_ERR_INVALID_ARG for a limit outside that range. */
+DORA_API int dora_selftest_timeout(int64_t limit_cycles, void* stream);
+
 /* Number of SMs the persistent kernels size their grids to on the current
  * device (the grid is a multiple of this count).  Returns 0 when no device. */
 DORA_API int dora_num_sms(void);

@@ -76,6 +76,13 @@ def test_norm_argument_errors(lib):
     assert _norm(lib, d_out=0) == D.DORA_OK  # nothing to do, nothing launched
 
 
+def test_selftest_timeout_argument_errors(lib):
+    # rejected on the host before any device work
+    assert lib.dora_selftest_timeout(0, None) == D.DORA_ERR_INVALID_ARG
+    assert lib.dora_selftest_timeout(-5, None) == D.DORA_ERR_INVALID_ARG
+    assert lib.dora_selftest_timeout(10**12, None) == D.DORA_ERR_INVALID_ARG
+
+
 def test_compose_argument_errors(lib):
     f = lib.dora_compose_fwd
     assert f(None, FAKE, FAKE, FAKE, 0.5, 4, 64, D.DORA_BF16, FAKE, None) == D.DORA_ERR_INVALID_ARG

@@ -57,6 +57,22 @@ def test_norm_bf16_small(shape, s):
     P.assert_norm_close(n, _oracle_norm(W, A, B, s), torch.bfloat16)
 
 
+def test_bounded_wait_timeout_is_reported_and_the_context_survives():
+    """A bounded wait that runs out (on an mbarrier nothing completes) records
+    DORA_ERR_TIMEOUT; the host reads and clears it, and the next call works."""
+    torch.cuda.synchronize()
+    assert D.dora_device_status() == D.DORA_OK
+    D.dora_selftest_timeout(2_000_000)  # about a millisecond
+    assert D.dora_device_status() == D.DORA_ERR_TIMEOUT
+    assert D.dora_device_status() == D.DORA_OK  # read-and-clear
+    wl = _wl(384, 640, 256)
+    W, A, B, _ = wlmod.make_weights(wl, DEV)
+    n = D.dora_factored_norm(W, A, B, wl.s)
+    torch.cuda.synchronize()
+    assert D.dora_device_status() == D.DORA_OK
+    P.assert_norm_close(n, _oracle_norm(W, A, B, wl.s), torch.bfloat16)
+
+
 def test_norm_bf16_s_zero_and_b_zero():
     wl = _wl(300, 256, 32)
     W, A, B, _ = wlmod.make_weights(wl, DEV)
