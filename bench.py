@@ -212,8 +212,43 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- end to end through the Python API with pinned host buffers
     e2e = run_e2e(args, D, dev, wl, W, A, B, m, base, lora, dy, n, y, d_base, d_lora, d_m, ws_n, ws_b, world)
+    dense = run_dense_comparator(D, dev, W, A, B, s, ws_n) if rank == 0 else None
     return dict(t_total=t_total, t_norm=t_norm, t_fwd=t_fwd, t_bwd=t_bwd, clocks=clocks, status=status, e2e=e2e,
-                wl=wl)
+                wl=wl, dense=dense)
+
+
+def run_dense_comparator(D, dev, W, A, B, s, ws_n, reps=10):
+    """Context, not our path: the row norm as the frameworks the pages survey
+    compute it, by materialising the dense [d_out, d_in] product B A in the
+    weight dtype (torch matmul, i.e. cuBLAS) and taking ||W + s B A||_row.
+    Returns its time and transient memory beside the factored norm's."""
+    def dense():
+        return torch.linalg.vector_norm((W + s * (B @ A)).float(), dim=1)
+
+    def timed(f):
+        for _ in range(3):
+            f()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            f()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps * 1e3
+
+    n = torch.empty(W.shape[0], dtype=torch.float32, device=dev)
+    t_dense = timed(dense)
+    t_factored = timed(lambda: D.dora_factored_norm(W, A, B, s, n_out=n, workspace=ws_n))
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats(dev)
+    before = torch.cuda.memory_allocated(dev)
+    dense()
+    torch.cuda.synchronize()
+    dense_peak = torch.cuda.max_memory_allocated(dev) - before
+    return {"what": "row norm by materialising B A (torch matmul, bf16) vs the factored norm; context only",
+            "dense_time_us": t_dense, "factored_time_us": t_factored,
+            "dense_transient_bytes": dense_peak, "factored_workspace_bytes": ws_n.numel()}
 
 
 def run_e2e(args, D, dev, wl, W, A, B, m, base, lora, dy, n, y, d_base, d_lora, d_m, ws_n, ws_b, world):
@@ -413,6 +448,8 @@ def build_line(args, res, N, peaks, peak_src, traffic, cpu):
         "clocks": res["clocks"],
         "device_status": res["status"],
     }
+    if res.get("dense") is not None:
+        line["dense_comparator"] = res["dense"]
     return line
 
 

@@ -281,6 +281,8 @@ __global__ void __launch_bounds__(kNormThreads, 1)
         record_timeout(a.status, abort_flag);
         ok = false;
       };
+      const uint64_t desc0 = sw128_kmajor_desc(base_s);
+      const uint64_t desc_step = a.stage_bytes >> 4;
       UnitIter x;
       int n_cur = -1;
       uint32_t idesc0 = 0, idesc1 = 0;
@@ -302,15 +304,21 @@ __global__ void __launch_bounds__(kNormThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t sW = base_s + stage * a.stage_bytes;
-        const uint64_t adesc = sw128_kmajor_desc(sW);
-        const uint64_t bdesc = sw128_kmajor_desc(sW + kBoxBytes);
+        // the stage's descriptors differ from stage 0's only in the start
+        // address field; +32 bytes along K inside the swizzled row is +2
+        const uint64_t adesc = desc0 + static_cast<uint64_t>(stage) * desc_step;
+        const uint64_t bdesc = adesc + (kBoxBytes >> 4);
+        const uint32_t acc0 = x.seg_first ? 0u : 1u;
+        if (idesc1) {
 #pragma unroll
-        for (int k = 0; k < kBK / 16; ++k) {
-          // +32 bytes along K inside the swizzled row is +2 in the 16-byte address field
-          const uint32_t acc = (x.seg_first && k == 0) ? 0u : 1u;
-          mma_bf16(tmem, adesc + 2 * k, bdesc + 2 * k, idesc0, acc);
-          if (idesc1) mma_bf16(tmem + 256, adesc + 2 * k, bdesc + (256 * 128 >> 4) + 2 * k, idesc1, acc);
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint32_t acc = k == 0 ? acc0 : 1u;
+            mma_bf16(tmem, adesc + 2 * k, bdesc + 2 * k, idesc0, acc);
+            mma_bf16(tmem + 256, adesc + 2 * k, bdesc + (256 * 128 >> 4) + 2 * k, idesc1, acc);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) mma_bf16(tmem, adesc + 2 * k, bdesc + 2 * k, idesc0, k == 0 ? acc0 : 1u);
         }
         mma_commit(&empty[stage]);
         advance();
