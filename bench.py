@@ -213,8 +213,9 @@ def run_ours(args, rank, world, local_rank):
     # ---- end to end through the Python API with pinned host buffers
     e2e = run_e2e(args, D, dev, wl, W, A, B, m, base, lora, dy, n, y, d_base, d_lora, d_m, ws_n, ws_b, world)
     dense = run_dense_comparator(D, dev, W, A, B, s, ws_n) if rank == 0 else None
+    batched = run_batched_context(D, dev) if rank == 0 else None
     return dict(t_total=t_total, t_norm=t_norm, t_fwd=t_fwd, t_bwd=t_bwd, clocks=clocks, status=status, e2e=e2e,
-                wl=wl, dense=dense)
+                wl=wl, dense=dense, batched=batched)
 
 
 def run_dense_comparator(D, dev, W, A, B, s, ws_n, reps=10):
@@ -249,6 +250,57 @@ def run_dense_comparator(D, dev, W, A, B, s, ws_n, reps=10):
     return {"what": "row norm by materialising B A (torch matmul, bf16) vs the factored norm; context only",
             "dense_time_us": t_dense, "factored_time_us": t_factored,
             "dense_transient_bytes": dense_peak, "factored_workspace_bytes": ws_n.numel()}
+
+
+# the seven adapted projections of one decoder block of an 8B-class model
+# (q, k, v, o, gate, up, down) as (d_out, d_in)
+BLOCK_SHAPES = [(4096, 4096), (1024, 4096), (1024, 4096), (4096, 4096), (14336, 4096), (14336, 4096), (4096, 14336)]
+
+
+def run_batched_context(D, dev, blocks=16, r=384, s=0.5, reps=3):
+    """Context for the many-module path: the norms of every adapted module
+    of `blocks` decoder blocks (7 modules each, bf16, r = 384, synthetic),
+    computed by one dora_factored_norm_batched call versus one
+    dora_factored_norm call per module, both timed with CUDA events."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(1234)
+    mods = []
+    for _ in range(blocks):
+        for d_out, d_in in BLOCK_SHAPES:
+            W = (torch.randn(d_out, d_in, generator=g, device=dev) * 0.02).bfloat16()
+            A = ((torch.rand(r, d_in, generator=g, device=dev) * 2 - 1) / d_in ** 0.5).bfloat16()
+            B = (torch.randn(d_out, r, generator=g, device=dev) * 0.002).bfloat16()
+            mods.append((W, A, B, s))
+    outs = [torch.empty(m[0].shape[0], dtype=torch.float32, device=dev) for m in mods]
+    ws_b = torch.empty(D.dora_factored_norm_batched_workspace_size(mods), dtype=torch.uint8, device=dev)
+    ws_1 = torch.empty(max(D.dora_factored_norm_workspace_size(m[0].shape[0], m[0].shape[1], r) for m in mods),
+                       dtype=torch.uint8, device=dev)
+
+    def batched():
+        D.dora_factored_norm_batched(mods, n_outs=outs, workspace=ws_b)
+
+    def one_by_one():
+        for (W, A, B, sm), n in zip(mods, outs):
+            D.dora_factored_norm(W, A, B, sm, n_out=n, workspace=ws_1)
+
+    def timed(f):
+        f()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            f()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps * 1e3
+
+    t_b, t_1 = timed(batched), timed(one_by_one)
+    F = sum(norm_flops(m[0].shape[0], m[0].shape[1], r) for m in mods)
+    return {"what": f"norms of {len(mods)} modules ({blocks} decoder blocks x q,k,v,o,gate,up,down of an "
+                    f"8B-class model, r = {r}, bf16, synthetic): one batched call vs one call per module",
+            "modules": len(mods), "batched_us": t_b, "one_by_one_us": t_1,
+            "batched_tflops": F / (t_b * 1e-6) / 1e12, "one_by_one_tflops": F / (t_1 * 1e-6) / 1e12,
+            "device_status": D.dora_device_status()}
 
 
 def run_e2e(args, D, dev, wl, W, A, B, m, base, lora, dy, n, y, d_base, d_lora, d_m, ws_n, ws_b, world):
@@ -450,6 +502,8 @@ def build_line(args, res, N, peaks, peak_src, traffic, cpu):
     }
     if res.get("dense") is not None:
         line["dense_comparator"] = res["dense"]
+    if res.get("batched") is not None:
+        line["many_modules"] = res["batched"]
     return line
 
 

@@ -11,12 +11,14 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <vector>
 #include <mutex>
 
 #include "../../include/dora.h"
 #include "compose.cuh"
 #include "norm_simt.cuh"
 #include "norm_tc.cuh"
+#include "norm_batched.cuh"
 
 namespace dora {
 
@@ -68,6 +70,11 @@ int device_info(DeviceInfo** out) {
     if (cudaFuncSetAttribute(norm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin) != cudaSuccess)
       return DORA_ERR_CUDA;
     if (cudaFuncSetAttribute(gram_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin) != cudaSuccess)
+      return DORA_ERR_CUDA;
+    if (cudaFuncSetAttribute(norm_batched_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(gram_batched_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin) !=
+            cudaSuccess)
       return DORA_ERR_CUDA;
     if (!g_encode) {
       void* fn = nullptr;
@@ -241,6 +248,136 @@ int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_
   return launch_error();
 }
 
+// Argument checks of one factored norm, workspace aside.
+int norm_arg_status(const void* W, const void* A, const void* B, int64_t d_out, int64_t d_in, int64_t r, dora_dtype dt,
+                    const float* n_out) {
+  if (dt != DORA_BF16 && dt != DORA_F32) return DORA_ERR_UNSUPPORTED;
+  if (d_out < 0 || d_in < 0 || r < 0) return DORA_ERR_INVALID_ARG;
+  if (d_out > INT32_MAX / 2 || d_in > INT32_MAX / 2 || r > kMaxRank) return DORA_ERR_UNSUPPORTED;
+  if (d_out == 0) return DORA_OK;
+  if (!n_out || (d_in > 0 && !W) || (r > 0 && d_in > 0 && (!A || !B))) return DORA_ERR_INVALID_ARG;
+  if (!aligned(n_out, 4)) return DORA_ERR_UNSUPPORTED;
+  if (dt == DORA_BF16) {
+    if (d_in > 0 && (d_in % 8 != 0 || r % 16 != 0)) return DORA_ERR_UNSUPPORTED;
+    if (!aligned(W, 16) || !aligned(A, 16) || !aligned(B, 16)) return DORA_ERR_UNSUPPORTED;
+  } else {
+    if (!aligned(W, 4) || !aligned(A, 4) || !aligned(B, 4)) return DORA_ERR_UNSUPPORTED;
+  }
+  return DORA_OK;
+}
+
+// ------------------------------------------------------- batched norms
+// Modules that share the two batched launches: bf16, 16 <= r <= 512 (one
+// TMEM chunk), something to compute.
+bool batchable(const dora_norm_problem& q, dora_dtype dt) {
+  return dt == DORA_BF16 && q.d_out > 0 && q.d_in > 0 && q.r >= 16 && q.r <= 512 && q.r % 16 == 0;
+}
+
+struct BatchLayout {
+  std::vector<int> batched, single;  // problem indices on each path
+  std::vector<size_t> off_gs;        // per batched problem: its G' in the workspace
+  size_t off_items = 0, off_gitems = 0, off_single = 0, single_bytes = 0, total = 0;
+  int n_items = 0, n_gitems = 0;
+  uint32_t stage_bytes = 0;
+};
+
+int batch_layout(const dora_norm_problem* q, int count, dora_dtype dt, BatchLayout* L) {
+  if (dt != DORA_BF16 && dt != DORA_F32) return DORA_ERR_UNSUPPORTED;
+  if (count < 0 || (count > 0 && !q)) return DORA_ERR_INVALID_ARG;
+  for (int i = 0; i < count; ++i) {
+    if (q[i].d_out < 0 || q[i].d_in < 0 || q[i].r < 0) return DORA_ERR_INVALID_ARG;
+    if (batchable(q[i], dt)) {
+      L->batched.push_back(i);
+      L->n_items += static_cast<int>(cdiv(q[i].d_out, kBM));
+      const int nt = static_cast<int>(cdiv(q[i].r, kBoxRows));
+      L->n_gitems += nt * nt;
+      L->stage_bytes = std::max<uint32_t>(L->stage_bytes, kBoxBytes * (1 + nt));
+    } else {
+      L->single.push_back(i);
+      L->single_bytes = std::max(L->single_bytes, dora_factored_norm_workspace_size(q[i].d_out, q[i].d_in, q[i].r, dt));
+    }
+  }
+  size_t off = align_up(L->batched.size() * sizeof(BatchDesc), 256);
+  L->off_items = off;
+  off = align_up(off + static_cast<size_t>(L->n_items) * sizeof(BatchItem), 256);
+  L->off_gitems = off;
+  off = align_up(off + static_cast<size_t>(L->n_gitems) * sizeof(BatchItem), 256);
+  for (int i : L->batched) {
+    L->off_gs.push_back(off);
+    off = align_up(off + static_cast<size_t>(q[i].r) * q[i].r * 2, 256);
+  }
+  L->off_single = off;
+  L->total = off + L->single_bytes;
+  return DORA_OK;
+}
+
+int norm_batched(const dora_norm_problem* q, const BatchLayout& L, uint8_t* ws, cudaStream_t st, DeviceInfo* dev) {
+  const size_t nb = L.batched.size();
+  // the descriptor table and both work lists, built here and copied in one go
+  std::vector<uint8_t> host(L.off_gs.empty() ? L.off_gitems : L.off_gs[0]);
+  BatchDesc* descs = reinterpret_cast<BatchDesc*>(host.data());
+  BatchItem* items = reinterpret_cast<BatchItem*>(host.data() + L.off_items);
+  BatchItem* gitems = reinterpret_cast<BatchItem*>(host.data() + L.off_gitems);
+  int ni = 0, ng = 0;
+  for (size_t j = 0; j < nb; ++j) {
+    const dora_norm_problem& p = q[L.batched[j]];
+    BatchDesc& d = descs[j];
+    std::memset(&d, 0, sizeof(d));
+    __nv_bfloat16* gs = reinterpret_cast<__nv_bfloat16*>(ws + L.off_gs[j]);
+    if (make_map(&d.tmW, p.W, p.d_out, p.d_in) || make_map(&d.tmA, p.A, p.r, p.d_in) ||
+        make_map(&d.tmB, p.B, p.d_out, p.r) || make_map(&d.tmG, gs, p.r, p.r))
+      return DORA_ERR_CUDA;
+    d.n_out = p.n_out;
+    d.gs = gs;
+    d.d_out = static_cast<int>(p.d_out);
+    d.d_in = static_cast<int>(p.d_in);
+    d.r = static_cast<int>(p.r);
+    d.kb_main = static_cast<int>(cdiv(p.d_in, kBK));
+    d.kb_total = d.kb_main + static_cast<int>(cdiv(p.r, kBK));
+    d.two_s = 2.0f * p.s;
+    d.half_s = 0.5f * p.s;
+    for (int t = 0; t < cdiv(p.d_out, kBM); ++t) items[ni++] = BatchItem{static_cast<int>(j), t};
+    const int nt = static_cast<int>(cdiv(p.r, kBoxRows));
+    for (int t = 0; t < nt * nt; ++t) gitems[ng++] = BatchItem{static_cast<int>(j), t};
+  }
+  // longest items first, dealt round-robin over the persistent grid
+  auto cost = [&](const BatchItem& it) {
+    const BatchDesc& d = descs[it.prob];
+    return static_cast<long long>(d.kb_total) * (1 + cdiv(d.r, kBoxRows));
+  };
+  std::stable_sort(items, items + ni, [&](const BatchItem& x, const BatchItem& y) { return cost(x) > cost(y); });
+  if (cudaMemcpyAsync(ws, host.data(), host.size(), cudaMemcpyHostToDevice, st) != cudaSuccess) return DORA_ERR_CUDA;
+
+  const BatchDesc* d_descs = reinterpret_cast<const BatchDesc*>(ws);
+  const size_t gram_smem = kGramStages * kGramStageBytes + (2 * kGramStages + 1) * 8 + 16 + 1024;
+  gram_batched_kernel<<<ng, kNormThreads, gram_smem, st>>>(d_descs, reinterpret_cast<const BatchItem*>(ws + L.off_gitems),
+                                                          kWaitLimitCycles, dev->status);
+  if (launch_error()) return DORA_ERR_CUDA;
+
+  BatchNormArgs a{};
+  a.n_items = ni;
+  a.stage_bytes = L.stage_bytes;
+  const size_t fixed = 1024 + 64 + 16;
+  a.stages = static_cast<int>(std::min<size_t>(kMaxStages, (dev->smem_optin - fixed) / (a.stage_bytes + 16)));
+  if (a.stages < 2) return DORA_ERR_UNSUPPORTED;
+  a.wait_limit = kWaitLimitCycles;
+  a.status = dev->status;
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.stream = st;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(std::min<long long>({static_cast<long long>(dev->num_sms), ni, kMaxGrid})));
+  cfg.blockDim = dim3(kNormThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(a.stages) * a.stage_bytes + (2 * a.stages + 3) * 8 + 16 + 1024;
+  if (cudaLaunchKernelEx(&cfg, norm_batched_kernel, d_descs, reinterpret_cast<const BatchItem*>(ws + L.off_items), a) !=
+      cudaSuccess)
+    return DORA_ERR_CUDA;
+  return launch_error();
+}
+
 }  // namespace
 }  // namespace dora
 
@@ -270,22 +407,12 @@ size_t dora_factored_norm_workspace_size(int64_t d_out, int64_t d_in, int64_t r,
 
 int dora_factored_norm(const void* W, const void* A, const void* B, int64_t d_out, int64_t d_in, int64_t r, float s,
                        dora_dtype dt, float* n_out, void* workspace, size_t workspace_bytes, void* stream) {
-  if (dt != DORA_BF16 && dt != DORA_F32) return DORA_ERR_UNSUPPORTED;
-  if (d_out < 0 || d_in < 0 || r < 0) return DORA_ERR_INVALID_ARG;
-  if (d_out > INT32_MAX / 2 || d_in > INT32_MAX / 2 || r > kMaxRank) return DORA_ERR_UNSUPPORTED;
-  if (d_out == 0) return DORA_OK;
-  if (!n_out || (d_in > 0 && !W) || (r > 0 && d_in > 0 && (!A || !B))) return DORA_ERR_INVALID_ARG;
-  if (!aligned(n_out, 4)) return DORA_ERR_UNSUPPORTED;
+  const int arg = norm_arg_status(W, A, B, d_out, d_in, r, dt, n_out);
+  if (arg != DORA_OK || d_out == 0) return arg;
   const size_t need = dora_factored_norm_workspace_size(d_out, d_in, r, dt);
   const bool trivial = (d_in == 0);
   if (!trivial && (!workspace || workspace_bytes < need)) return DORA_ERR_WORKSPACE;
   if (!trivial && !aligned(workspace, 256)) return DORA_ERR_UNSUPPORTED;
-  if (dt == DORA_BF16) {
-    if (!trivial && (d_in % 8 != 0 || r % 16 != 0)) return DORA_ERR_UNSUPPORTED;
-    if (!aligned(W, 16) || !aligned(A, 16) || !aligned(B, 16)) return DORA_ERR_UNSUPPORTED;
-  } else {
-    if (!aligned(W, 4) || !aligned(A, 4) || !aligned(B, 4)) return DORA_ERR_UNSUPPORTED;
-  }
   DeviceInfo* dev = nullptr;
   if (device_info(&dev)) return DORA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -432,6 +559,42 @@ int dora_compose_bwd(const void* dy, const void* base_out, const void* lora_out,
         static_cast<const float*>(dy), static_cast<const float*>(base_out), static_cast<const float*>(lora_out), m, n,
         s, tokens, nvec, d_out, static_cast<float*>(d_base), static_cast<float*>(d_lora), part, cnt, d_m, rows);
   return launch_error();
+}
+
+size_t dora_factored_norm_batched_workspace_size(const dora_norm_problem* problems, int count, dora_dtype dt) {
+  BatchLayout L;
+  if (batch_layout(problems, count, dt, &L) != DORA_OK) return 0;
+  return std::max<size_t>(L.total, 256);
+}
+
+int dora_factored_norm_batched(const dora_norm_problem* problems, int count, dora_dtype dt, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  BatchLayout L;
+  const int lay = batch_layout(problems, count, dt, &L);
+  if (lay != DORA_OK) return lay;
+  // every module's arguments are checked before anything is launched
+  for (int i = 0; i < count; ++i) {
+    const dora_norm_problem& q = problems[i];
+    const int arg = norm_arg_status(q.W, q.A, q.B, q.d_out, q.d_in, q.r, dt, q.n_out);
+    if (arg != DORA_OK) return arg;
+  }
+  if (count == 0) return DORA_OK;
+  if (!workspace || workspace_bytes < L.total) return DORA_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return DORA_ERR_UNSUPPORTED;
+  DeviceInfo* dev = nullptr;
+  if (device_info(&dev)) return DORA_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (!L.batched.empty()) {
+    const int rc = norm_batched(problems, L, ws, static_cast<cudaStream_t>(stream), dev);
+    if (rc != DORA_OK) return rc;
+  }
+  for (int i : L.single) {
+    const dora_norm_problem& q = problems[i];
+    const int rc = dora_factored_norm(q.W, q.A, q.B, q.d_out, q.d_in, q.r, q.s, dt, q.n_out, ws + L.off_single,
+                                      L.single_bytes, stream);
+    if (rc != DORA_OK) return rc;
+  }
+  return DORA_OK;
 }
 
 int dora_device_status(void* stream) {

@@ -119,6 +119,13 @@ __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int x
                : "memory");
 }
 
+// Makes a tensor map that lives in global memory (written by a copy before
+// this launch) visible to this thread's later TMA operations that use it.
+__device__ __forceinline__ void tensormap_acquire(const CUtensorMap* map) {
+  asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(reinterpret_cast<uint64_t>(map))
+               : "memory");
+}
+
 // 2-D tiled load of one box into shared memory; completion is signalled on
 // `bar` as transaction bytes.  x is the innermost (contiguous) coordinate.
 __device__ __forceinline__ void tma_load_2d(uint32_t smem_dst, const CUtensorMap* map, uint64_t* bar, int x,

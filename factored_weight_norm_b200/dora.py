@@ -27,8 +27,19 @@ DORA_ERR_WORKSPACE = 3
 DORA_ERR_CUDA = 4
 DORA_ERR_TIMEOUT = 5
 
-# every symbol include/dora.h declares, with its ctypes signature
 _c_void_p, _i64, _f32, _size = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+
+
+class NormProblem(ctypes.Structure):
+    """dora_norm_problem of include/dora.h."""
+
+    _fields_ = [("W", _c_void_p), ("A", _c_void_p), ("B", _c_void_p), ("d_out", _i64), ("d_in", _i64),
+                ("r", _i64), ("s", _f32), ("n_out", _c_void_p)]
+
+
+_problems_p = ctypes.POINTER(NormProblem)
+
+# every symbol include/dora.h declares, with its ctypes signature
 SIGNATURES = {
     "dora_factored_norm_workspace_size": (_size, [_i64, _i64, _i64, ctypes.c_int]),
     "dora_factored_norm": (
@@ -54,6 +65,8 @@ SIGNATURES = {
     "dora_device_status": (ctypes.c_int, [_c_void_p]),
     "dora_num_sms": (ctypes.c_int, []),
     "dora_selftest_timeout": (ctypes.c_int, [_i64, _c_void_p]),
+    "dora_factored_norm_batched_workspace_size": (_size, [_problems_p, ctypes.c_int, ctypes.c_int]),
+    "dora_factored_norm_batched": (ctypes.c_int, [_problems_p, ctypes.c_int, ctypes.c_int, _c_void_p, _size, _c_void_p]),
 }
 
 _lib = None
@@ -165,6 +178,48 @@ def dora_factored_norm(W, A, B, s: float, n_out=None, workspace=None, stream=Non
     )
     _check(st, "dora_factored_norm")
     return n_out
+
+
+def _problem_array(modules, n_outs):
+    arr = (NormProblem * len(modules))()
+    for i, ((W, A, B, s), n) in enumerate(zip(modules, n_outs)):
+        _dense_cuda(W, A, B, n)
+        d_out, d_in = W.shape
+        r = A.shape[0]
+        if A.shape != (r, d_in) or B.shape != (d_out, r) or n.shape != (d_out,):
+            raise ValueError(f"module {i}: shape mismatch: W {tuple(W.shape)}, A {tuple(A.shape)}, B {tuple(B.shape)}")
+        if not (W.dtype == A.dtype == B.dtype) or n.dtype != torch.float32:
+            raise TypeError(f"module {i}: W, A, B share one dtype; n is fp32")
+        arr[i] = NormProblem(W.data_ptr(), A.data_ptr(), B.data_ptr(), d_out, d_in, r, float(s), n.data_ptr())
+    return arr
+
+
+def dora_factored_norm_batched_workspace_size(modules, dtype: torch.dtype = torch.bfloat16) -> int:
+    """modules: sequence of (W, A, B, s) with W [d_out, d_in], A [r, d_in], B [d_out, r]."""
+    n_outs = [torch.empty(W.shape[0], dtype=torch.float32, device=W.device) for (W, _, _, _) in modules]
+    arr = _problem_array(modules, n_outs)
+    return int(lib().dora_factored_norm_batched_workspace_size(arr, len(modules), _dt(torch.empty(0, dtype=dtype))))
+
+
+def dora_factored_norm_batched(modules, n_outs=None, workspace=None, stream=None):
+    """The factored row norms of many modules at once; modules: sequence of
+    (W, A, B, s).  Returns the list of fp32 n tensors."""
+    modules = list(modules)
+    if not modules:
+        return []
+    dev = modules[0][0].device
+    if n_outs is None:
+        n_outs = [torch.empty(W.shape[0], dtype=torch.float32, device=dev) for (W, _, _, _) in modules]
+    arr = _problem_array(modules, n_outs)
+    dt = _dt(modules[0][0])
+    need = int(lib().dora_factored_norm_batched_workspace_size(arr, len(modules), dt))
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    _dense_cuda(workspace)
+    st = lib().dora_factored_norm_batched(arr, len(modules), dt, _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "dora_factored_norm_batched")
+    return n_outs
 
 
 def dora_compose_fwd(base_out, lora_out, m, n, s: float, y=None, stream=None):

@@ -77,6 +77,39 @@ DORA_API int dora_factored_norm(const void* W, const void* A, const void* B, int
                        float s, dora_dtype dt, float* n_out, void* workspace, size_t workspace_bytes,
                        void* stream);
 
+/* One adapted module for dora_factored_norm_batched: the arguments of
+ * dora_factored_norm for that module (device pointers, row-major layouts as
+ * above; n_out is overwritten). */
+typedef struct {
+  const void* W;
+  const void* A;
+  const void* B;
+  int64_t d_out, d_in, r;
+  float s;
+  float* n_out;
+} dora_norm_problem;
+
+/* Bytes of workspace dora_factored_norm_batched needs for these modules
+ * (`problems`: host array of `count`); 0 for invalid arguments. */
+DORA_API size_t dora_factored_norm_batched_workspace_size(const dora_norm_problem* problems, int count, dora_dtype dt);
+
+/* The factored row norms of `count` adapted modules at once (Scaling DoRA,
+ * Abstract: models carry "hundreds of adapted modules"), each computing
+ * exactly what dora_factored_norm computes for it.  `problems` is a host
+ * array, read during the call only.  Modules with bf16 weights and
+ * 16 <= r <= 512 share two launches: every 128 x 128 tile of every module's
+ * Gram matrix, then one persistent GEMM over a work list of (module, 128-row
+ * tile) items, each item finishing its rows' norms; the other modules are
+ * computed one by one as by dora_factored_norm, on the same stream.
+ * Every module's arguments are checked (as dora_factored_norm checks them)
+ * before anything is launched.  workspace: device buffer of at least
+ * dora_factored_norm_batched_workspace_size() bytes, 256-byte aligned,
+ * contents ignored on entry; it holds the modules' descriptor table (copied
+ * from the host with cudaMemcpyAsync), their G' = (s/2) G and the scratch of
+ * the one-by-one modules.  Asynchronous on `stream`; count == 0 does nothing. */
+DORA_API int dora_factored_norm_batched(const dora_norm_problem* problems, int count, dora_dtype dt, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+
 /* Fused DoRA compose, one pass (Scaling DoRA, Abstract: the four-kernel
  * composition collapsed into a single pass, in a numerically stable form for
  * the near-unity regime):

@@ -83,6 +83,42 @@ def test_selftest_timeout_argument_errors(lib):
     assert lib.dora_selftest_timeout(10**12, None) == D.DORA_ERR_INVALID_ARG
 
 
+def _problems(*specs):
+    arr = (D.NormProblem * len(specs))()
+    for i, sp in enumerate(specs):
+        q = dict(W=FAKE.value, A=FAKE.value, B=FAKE.value, d_out=256, d_in=128, r=16, s=0.5, n_out=FAKE.value)
+        q.update(sp)
+        arr[i] = D.NormProblem(q["W"], q["A"], q["B"], q["d_out"], q["d_in"], q["r"], q["s"], q["n_out"])
+    return arr
+
+
+def test_batched_argument_errors(lib):
+    f, size = lib.dora_factored_norm_batched, lib.dora_factored_norm_batched_workspace_size
+    good = _problems({}, {"r": 384, "d_out": 1000})
+    need = size(good, 2, D.DORA_BF16)
+    assert need > 0
+    assert f(None, 0, D.DORA_BF16, None, 0, None) == D.DORA_OK  # nothing to do
+    assert f(None, 2, D.DORA_BF16, None, 0, None) == D.DORA_ERR_INVALID_ARG
+    assert size(None, -1, D.DORA_BF16) == 0
+    assert f(good, 2, 7, FAKE, need, None) == D.DORA_ERR_UNSUPPORTED
+    # every module is checked before anything is launched
+    assert f(_problems({}, {"d_out": -1}), 2, D.DORA_BF16, FAKE, 1 << 30, None) == D.DORA_ERR_INVALID_ARG
+    assert f(_problems({}, {"W": None}), 2, D.DORA_BF16, FAKE, 1 << 30, None) == D.DORA_ERR_INVALID_ARG
+    assert f(_problems({"d_in": 100}), 1, D.DORA_BF16, FAKE, 1 << 30, None) == D.DORA_ERR_UNSUPPORTED
+    assert f(_problems({"r": 24}), 1, D.DORA_BF16, FAKE, 1 << 30, None) == D.DORA_ERR_UNSUPPORTED
+    assert f(good, 2, D.DORA_BF16, None, 0, None) == D.DORA_ERR_WORKSPACE
+    assert f(good, 2, D.DORA_BF16, FAKE, need - 1, None) == D.DORA_ERR_WORKSPACE
+    assert f(good, 2, D.DORA_BF16, MISALIGNED, need, None) == D.DORA_ERR_UNSUPPORTED
+
+
+def test_batched_workspace_has_no_dense_term(lib):
+    # 64 modules of 8192 x 8192 at r = 384: the table, the work lists and each
+    # module's (s/2) G, nothing of size d_out x d_in
+    arr = _problems(*[{"d_out": 8192, "d_in": 8192, "r": 384}] * 64)
+    need = lib.dora_factored_norm_batched_workspace_size(arr, 64, D.DORA_BF16)
+    assert need < 64 * (384 * 384 * 2 + 4096) + (1 << 20)
+
+
 def test_compose_argument_errors(lib):
     f = lib.dora_compose_fwd
     assert f(None, FAKE, FAKE, FAKE, 0.5, 4, 64, D.DORA_BF16, FAKE, None) == D.DORA_ERR_INVALID_ARG
