@@ -27,7 +27,7 @@ the factored algorithm:
     W' = W + s * (B @ A)                  dense [d_out, d_in], fp64
     n_i = sqrt(sum_k W'_ik ** 2)          one norm per output channel
     g_i = m_i / n_i
-    y[t, i] = g_i * (base[t, i] + s * lora[t, i])
+    y[t, i] = g_i * (base[t, i] + s * lora[t, i])     (no bias; see below)
 
 Backward (the norm ``n`` is held constant, see ``compose_backward``) with an
 upstream gradient ``dy``:
@@ -52,7 +52,13 @@ Readings where the pages are silent (each also listed in the design notes):
   outputs the hot path is asked for.
 * No epsilon is invented: ``n_i^2`` is used as computed; ``n_i == 0`` gives
   IEEE inf/nan in ``g`` exactly as the definition does.
-* No bias term: ``base`` is bias-free.
+* Bias: the pages never mention one.  Where the adapted layer has a bias
+  ``b``, ``base`` is taken to be the frozen base layer's output ``x W^T + b``
+  (what a framework's base layer returns), and the magnitude rescaling acts
+  on the weight's product only, as the DoRA summary page's Method defines the
+  adapted weight ``m * V / ||V||``:  ``y = b + g * ((base - b) + s * lora)``.
+  ``bias=None`` (the default) is ``b = 0``.  The bias is frozen: no gradient
+  is returned for it.
 
 Every function takes float64 numpy arrays (callers round bf16 inputs first,
 then widen) and returns float64 results.  No blocking, fusion or reordering
@@ -120,38 +126,45 @@ def magnitude_scale(m, n) -> np.ndarray:
         return _f64(m) / _f64(n)
 
 
-def compose_forward(base, lora, m, n, s) -> np.ndarray:
-    """``y = g * (base + s * lora)`` broadcast over tokens.
+def _bias(bias, d_out) -> np.ndarray:
+    return np.zeros(d_out) if bias is None else _f64(bias)
+
+
+def compose_forward(base, lora, m, n, s, bias=None) -> np.ndarray:
+    """``y = b + g * ((base - b) + s * lora)`` broadcast over tokens.
 
     Scaling DoRA, Abstract: the DoRA composition of the base output, the LoRA
-    output and the magnitude rescaling.  ``base = x W^T`` and
-    ``lora = x A^T B^T`` (unscaled) are ``[tokens, d_out]``.
+    output and the magnitude rescaling.  ``base = x W^T + b`` and
+    ``lora = x A^T B^T`` (unscaled) are ``[tokens, d_out]``; ``bias`` is the
+    base layer's ``b`` (``None``: no bias), which the rescaling leaves alone.
     """
     base, lora = _f64(base), _f64(lora)
+    b = _bias(bias, base.shape[1])
     g = magnitude_scale(m, n)
-    return g[None, :] * (base + float(s) * lora)
+    return b[None, :] + g[None, :] * ((base - b[None, :]) + float(s) * lora)
 
 
-def compose_backward(dy, base, lora, m, n, s):
-    """Gradients of ``y = (m / n) * (base + s * lora)`` with ``n`` constant.
+def compose_backward(dy, base, lora, m, n, s, bias=None):
+    """Gradients of ``y = b + (m / n) * ((base - b) + s * lora)``, ``n`` constant.
 
     Returns ``(d_base, d_lora, d_m)``:
       d_base = g * dy,  d_lora = s * g * dy,
-      d_m_i  = sum_t dy[t, i] * (base[t, i] + s * lora[t, i]) / n_i.
+      d_m_i  = sum_t dy[t, i] * ((base[t, i] - b_i) + s * lora[t, i]) / n_i.
     Chain rule on the forward definition above (Scaling DoRA, Abstract,
-    "gradient computation"), with the norm detached.
+    "gradient computation"), with the norm detached and the bias frozen.
     """
     dy, base, lora = _f64(dy), _f64(base), _f64(lora)
     s = float(s)
+    b = _bias(bias, base.shape[1])
     g = magnitude_scale(m, n)
     d_base = g[None, :] * dy
     d_lora = s * g[None, :] * dy
     with np.errstate(divide="ignore", invalid="ignore"):
-        d_m = np.sum(dy * (base + s * lora), axis=0) / _f64(n)
+        d_m = np.sum(dy * ((base - b[None, :]) + s * lora), axis=0) / _f64(n)
     return d_base, d_lora, d_m
 
 
-def compose_backward_columns(dy, base, lora, m, n, s, cols) -> np.ndarray:
+def compose_backward_columns(dy, base, lora, m, n, s, cols, bias=None) -> np.ndarray:
     """``d_m`` of ``compose_backward`` for the output channels in ``cols``.
 
     ``dy``/``base``/``lora`` are the full ``[tokens, d_out]`` arrays (or any
@@ -161,5 +174,6 @@ def compose_backward_columns(dy, base, lora, m, n, s, cols) -> np.ndarray:
     dy_c = _f64(np.asarray(dy)[:, cols])
     base_c = _f64(np.asarray(base)[:, cols])
     lora_c = _f64(np.asarray(lora)[:, cols])
-    _, _, d_m = compose_backward(dy_c, base_c, lora_c, _f64(m)[cols], _f64(n)[cols], s)
+    b_c = None if bias is None else _f64(bias)[cols]
+    _, _, d_m = compose_backward(dy_c, base_c, lora_c, _f64(m)[cols], _f64(n)[cols], s, bias=b_c)
     return d_m

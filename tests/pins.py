@@ -22,7 +22,11 @@ Method):
 * derivatives      - central finite differences and fp64 torch.autograd of
                      the forward definition with n held constant;
 * hand-worked      - small integer cases with exact answers worked by hand,
-                     stored in tests/golden/hand_cases.json.
+                     stored in tests/golden/hand_cases.json;
+* bias             - the compose form with a bias (base = x W^T + b) equals
+                     the adapted layer itself, x (diag(m / n) (W + sBA))^T + b
+                     with n from numpy.linalg.norm, and its d_m equals
+                     torch.autograd of that layer in m (n constant).
 """
 
 from __future__ import annotations
@@ -245,6 +249,43 @@ def pin_autograd(compose_backward, seed=5):
     assert np.max(np.abs(d_base - base.grad.numpy())) < 1e-14
     assert np.max(np.abs(d_lora - lora.grad.numpy())) < 1e-14
     assert np.max(np.abs(d_m - m.grad.numpy())) < 1e-12
+
+
+# ------------------------------------------------------------------ bias
+def pin_bias_layer(compose_forward, compose_backward, seed=6):
+    """DoRA summary page, Method: the adapted weight is m * V / ||V|| per output
+    channel, V = W + sBA; a bias b is added after the product and is not
+    rescaled.  A framework's base layer returns x W^T + b."""
+    import torch
+
+    rng = np.random.default_rng(seed)
+    T, d_in, d_out, r = 5, 7, 6, 3
+    x = rng.standard_normal((T, d_in))
+    W, A, B = tiny_case(rng, d_out, d_in, r)
+    b = rng.standard_normal(d_out)
+    dy = rng.standard_normal((T, d_out))
+    for s in (0.5, -1.5):
+        V = W + s * (B @ A)
+        n = np.linalg.norm(V, axis=1)
+        m = n * rng.uniform(0.8, 1.2, d_out)
+        y_layer = x @ ((m / n)[:, None] * V).T + b[None, :]
+        base = x @ W.T + b[None, :]
+        lora = (x @ A.T) @ B.T
+        y = compose_forward(base, lora, m, n, s, bias=b)
+        assert np.max(np.abs(y - y_layer)) < 1e-12 * (1 + np.max(np.abs(y_layer)))
+        # no bias and a zero bias are the same thing
+        z = np.zeros(d_out)
+        assert np.array_equal(compose_forward(base, lora, m, n, s), compose_forward(base, lora, m, n, s, bias=z))
+
+        mt = torch.tensor(m, dtype=torch.float64, requires_grad=True)
+        yt = torch.tensor(x) @ ((mt / torch.tensor(n))[:, None] * torch.tensor(V)).T + torch.tensor(b)[None, :]
+        yt.backward(torch.tensor(dy))
+        d_base, d_lora, d_m = compose_backward(dy, base, lora, m, n, s, bias=b)
+        assert np.max(np.abs(d_m - mt.grad.numpy())) < 1e-11 * (1 + np.max(np.abs(d_m)))
+        # the bias does not change the activation gradients
+        d_base0, d_lora0, _ = compose_backward(dy, base, lora, m, n, s)
+        assert np.array_equal(d_base, d_base0) and np.array_equal(d_lora, d_lora0)
+        assert np.max(np.abs(d_base - (m / n)[None, :] * dy)) < 1e-15 * (1 + np.max(np.abs(d_base)))
 
 
 # ------------------------------------------------------------ hand-worked

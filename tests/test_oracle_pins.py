@@ -1,5 +1,7 @@
 """The CPU oracle against what the pages and the mathematics fix (no GPU)."""
 
+import functools
+
 import numpy as np
 import pytest
 import torch
@@ -27,6 +29,10 @@ def test_compose_invariants():
 
 def test_finite_differences():
     pins.pin_finite_differences(oracle.compose_forward, oracle.compose_backward)
+
+
+def test_bias_layer():
+    pins.pin_bias_layer(oracle.compose_forward, oracle.compose_backward)
 
 
 def test_autograd():
@@ -141,6 +147,28 @@ def _m_drop_col(W, A, B, s):
     return np.sqrt(np.sum(Wp[:, :-1] ** 2, axis=1)) if Wp.shape[1] > 1 else np.zeros(Wp.shape[0])
 
 
+def _with_bias(f):
+    # a forward mutant that handles the bias correctly, so that its own
+    # defect is the one a pin has to catch
+    @functools.wraps(f)
+    def g(base, lora, m, n, s, bias=None):
+        if bias is None:
+            return f(base, lora, m, n, s)
+        b = np.asarray(bias, float)[None, :]
+        return b + f(np.asarray(base, float) - b, lora, m, n, s)
+
+    return g
+
+
+def _f_bias_not_removed(base, lora, m, n, s, bias=None):
+    return (np.asarray(m, float) / np.asarray(n, float))[None, :] * (np.asarray(base, float) + s * np.asarray(lora))
+
+
+def _f_bias_not_restored(base, lora, m, n, s, bias=None):
+    b = 0.0 if bias is None else np.asarray(bias, float)[None, :]
+    return (np.asarray(m, float) / np.asarray(n, float))[None, :] * (np.asarray(base, float) - b + s * np.asarray(lora))
+
+
 def _f_inverted(base, lora, m, n, s):
     return (np.asarray(n, float) / np.asarray(m, float))[None, :] * (base + s * np.asarray(lora))
 
@@ -158,8 +186,10 @@ def _f_axis(base, lora, m, n, s):
 
 
 def _bwd(variant):
-    def f(dy, base, lora, m, n, s):
+    def f(dy, base, lora, m, n, s, bias=None):
         dy, base, lora, m, n = (np.asarray(v, float) for v in (dy, base, lora, m, n))
+        if bias is not None and variant != "dm_bias_kept":
+            base = base - np.asarray(bias, float)[None, :]
         g = m / n
         d_base = g[None, :] * dy
         d_lora = s * g[None, :] * dy
@@ -192,6 +222,7 @@ def _run_all_pins(row_norm, fwd, bwd):
     pins.pin_finite_differences(fwd, bwd)
     pins.pin_autograd(bwd)
     pins.pin_hand_cases(row_norm, fwd, bwd)
+    pins.pin_bias_layer(fwd, bwd)
 
 
 def test_pins_pass_on_oracle():
@@ -199,25 +230,30 @@ def test_pins_pass_on_oracle():
 
 
 NORM_MUTANTS = [_m_drop_s, _m_sign, _m_s_squared, _m_column_norm, _m_no_sqrt, _m_index, _m_drop_col]
-FWD_MUTANTS = [_f_inverted, _f_no_s, _f_g_on_base_only, _f_axis]
-BWD_MUTANTS = [_bwd(v) for v in ("dm_no_div", "dm_no_lora", "dlora_no_s", "dbase_no_g", "dm_div_m", "dm_axis")]
+FWD_MUTANTS = [_with_bias(f) for f in (_f_inverted, _f_no_s, _f_g_on_base_only, _f_axis)] + [
+    _f_bias_not_removed,
+    _f_bias_not_restored,
+]
+BWD_MUTANTS = [
+    _bwd(v) for v in ("dm_no_div", "dm_no_lora", "dlora_no_s", "dbase_no_g", "dm_div_m", "dm_axis", "dm_bias_kept")
+]
 
 
 @pytest.mark.parametrize("mutant", NORM_MUTANTS, ids=lambda f: f.__name__)
 def test_norm_mutant_is_caught(mutant):
-    with pytest.raises(Exception):
+    with pytest.raises((AssertionError, ValueError)):
         _run_all_pins(mutant, oracle.compose_forward, oracle.compose_backward)
 
 
 @pytest.mark.parametrize("mutant", FWD_MUTANTS, ids=lambda f: f.__name__)
 def test_forward_mutant_is_caught(mutant):
-    with pytest.raises(Exception):
+    with pytest.raises((AssertionError, ValueError)):
         _run_all_pins(oracle.row_norm, mutant, oracle.compose_backward)
 
 
 @pytest.mark.parametrize("idx", range(len(BWD_MUTANTS)))
 def test_backward_mutant_is_caught(idx):
-    with pytest.raises(Exception):
+    with pytest.raises((AssertionError, ValueError)):
         _run_all_pins(oracle.row_norm, oracle.compose_forward, BWD_MUTANTS[idx])
 
 
