@@ -6,10 +6,12 @@
 //
 // Forward, per output channel i (fp32, never rounded to the activation type):
 //   g = m / n,  delta = (m - n) / n   (m - n is exact when m / n is in [1/2, 2])
-//   y = base + (delta * base + g * s * lora)        one final rounding
-// Backward with n constant:
-//   d_base = g * dy,  d_lora = (g * s) * dy,
-//   d_m    = (sum_t dy * (base + s * lora)) / n
+//   y = base + (delta * (base - b) + g * s * lora)  one final rounding
+// where b is the base layer's bias (0 without one): base = x W^T + b, and the
+// rescaling acts on the weight's product only, b + g * ((base - b) + s * lora).
+// Backward with n constant and b frozen:
+//   d_base = g * dy,  d_lora = s * (g * dy),
+//   d_m    = (sum_t dy * ((base - b) + s * lora)) / n
 //
 // Both kernels stream 16-byte vectors (8 bf16 or 4 fp32), coalesced along the
 // contiguous d_out axis; each thread keeps its channels' g / delta in
@@ -26,8 +28,23 @@ namespace dora {
 template <typename T, int VEC>
 struct VecIO;
 
+// load() widens at once; raw() / unpack() keep a vector packed (fewer
+// registers while several rows are in flight) and widen it at its use.
 template <>
 struct VecIO<__nv_bfloat16, 8> {
+  using Raw = uint4;
+  static __device__ __forceinline__ Raw raw(const __nv_bfloat16* p) { return ld_stream_u4(p); }
+  static __device__ __forceinline__ Raw raw_param(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+  static __device__ __forceinline__ void unpack(const Raw& u, float (&v)[8]) {
+    v[0] = bf16_lo(u.x);
+    v[1] = bf16_hi(u.x);
+    v[2] = bf16_lo(u.y);
+    v[3] = bf16_hi(u.y);
+    v[4] = bf16_lo(u.z);
+    v[5] = bf16_hi(u.z);
+    v[6] = bf16_lo(u.w);
+    v[7] = bf16_hi(u.w);
+  }
   static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[8]) {
     const uint4 u = ld_stream_u4(p);
     v[0] = bf16_lo(u.x);
@@ -55,6 +72,15 @@ struct VecIO<__nv_bfloat16, 8> {
 
 template <>
 struct VecIO<float, 4> {
+  using Raw = uint4;
+  static __device__ __forceinline__ Raw raw(const float* p) { return ld_stream_u4(p); }
+  static __device__ __forceinline__ Raw raw_param(const float* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+  static __device__ __forceinline__ void unpack(const Raw& u, float (&v)[4]) {
+    v[0] = __uint_as_float(u.x);
+    v[1] = __uint_as_float(u.y);
+    v[2] = __uint_as_float(u.z);
+    v[3] = __uint_as_float(u.w);
+  }
   static __device__ __forceinline__ void load(const float* p, float (&v)[4]) {
     const uint4 u = ld_stream_u4(p);
     v[0] = __uint_as_float(u.x);
@@ -70,26 +96,35 @@ struct VecIO<float, 4> {
 
 template <>
 struct VecIO<float, 1> {
+  using Raw = float;
+  static __device__ __forceinline__ Raw raw(const float* p) { return __ldg(p); }
+  static __device__ __forceinline__ Raw raw_param(const float* p) { return __ldg(p); }
+  static __device__ __forceinline__ void unpack(const Raw& u, float (&v)[1]) { v[0] = u; }
   static __device__ __forceinline__ void load(const float* p, float (&v)[1]) { v[0] = __ldg(p); }
   static __device__ __forceinline__ void store(float* p, const float (&v)[1]) { p[0] = v[0]; }
 };
 
+// One per-channel parameter of the activation type, widened to fp32.
+__device__ __forceinline__ float ld_param(const __nv_bfloat16* p) { return __bfloat162float(p[0]); }
+__device__ __forceinline__ float ld_param(const float* p) { return __ldg(p); }
+
 // ------------------------------------------------------------------ forward
 template <typename T, int VEC>
 __global__ void __launch_bounds__(256, 3) compose_fwd_kernel(const T* __restrict__ base, const T* __restrict__ lora,
-                                                          const float* __restrict__ m,
+                                                          const T* __restrict__ bias, const float* __restrict__ m,
                                                           const float* __restrict__ n, float s,
                                                           long long tokens, long long nvec, long long d_out,
                                                           T* __restrict__ y, long long rows_per_cta) {
   const long long v = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
   if (v >= nvec) return;
   const long long col = v * VEC;
-  float delta[VEC], gs[VEC];
+  float delta[VEC], gs[VEC], bb[VEC];
 #pragma unroll
   for (int e = 0; e < VEC; ++e) {
     const float mm = __ldg(m + col + e), nn = __ldg(n + col + e);
     delta[e] = (mm - nn) / nn;
     gs[e] = (mm / nn) * s;
+    bb[e] = bias ? ld_param(bias + col + e) : 0.f;
   }
   const long long row0 = blockIdx.y * rows_per_cta;
   const long long row1 = min(tokens, row0 + rows_per_cta);
@@ -106,7 +141,7 @@ __global__ void __launch_bounds__(256, 3) compose_fwd_kernel(const T* __restrict
     for (int k = 0; k < U; ++k) {
       float o[VEC];
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) o[e] = b[k][e] + fmaf(delta[e], b[k][e], gs[e] * l[k][e]);
+      for (int e = 0; e < VEC; ++e) o[e] = b[k][e] + fmaf(delta[e], b[k][e] - bb[e], gs[e] * l[k][e]);
       VecIO<T, VEC>::store(y + (row + k) * d_out + col, o);
     }
   }
@@ -115,7 +150,7 @@ __global__ void __launch_bounds__(256, 3) compose_fwd_kernel(const T* __restrict
     VecIO<T, VEC>::load(base + row * d_out + col, b);
     VecIO<T, VEC>::load(lora + row * d_out + col, l);
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) o[e] = b[e] + fmaf(delta[e], b[e], gs[e] * l[e]);
+    for (int e = 0; e < VEC; ++e) o[e] = b[e] + fmaf(delta[e], b[e] - bb[e], gs[e] * l[e]);
     VecIO<T, VEC>::store(y + row * d_out + col, o);
   }
 }
@@ -126,9 +161,12 @@ constexpr int kBwdVecs = 16;      // vectors (column groups) per CTA strip
 constexpr int kBwdSlots = 16;     // rows visited concurrently by one CTA
 constexpr int kBwdRows = 4;       // rows in flight per thread
 
-template <typename T, int VEC>
+// HAS_BIAS: a separate instantiation, so that the bias registers cost the
+// no-bias kernel nothing
+template <typename T, int VEC, bool HAS_BIAS>
 __global__ void __launch_bounds__(kBwdThreads, 2) compose_bwd_kernel(
-    const T* __restrict__ dy, const T* __restrict__ base, const T* __restrict__ lora, const float* __restrict__ m,
+    const T* __restrict__ dy, const T* __restrict__ base, const T* __restrict__ lora, const T* __restrict__ bias,
+    const float* __restrict__ m,
     const float* __restrict__ n, float s, long long tokens, long long nvec, long long d_out, T* __restrict__ d_base,
     T* __restrict__ d_lora, float* __restrict__ partial, int* __restrict__ counters, float* __restrict__ d_m,
     long long rows_per_chunk) {
@@ -141,42 +179,54 @@ __global__ void __launch_bounds__(kBwdThreads, 2) compose_bwd_kernel(
   const bool valid = v < nvec;
   const long long col = v * VEC;
 
-  float g[VEC], gs[VEC], acc[VEC];
+  // d_lora is formed as s * d_base (fp32) rather than from a second per-channel
+  // factor g * s: the registers go to the bias instead
+  // the bias stays packed in the activation type (half the registers for
+  // bf16) and is widened where it is used
+  using Raw = typename VecIO<T, VEC>::Raw;
+  float g[VEC], acc[VEC];
+  Raw bias_raw{};
 #pragma unroll
   for (int e = 0; e < VEC; ++e) {
     acc[e] = 0.f;
     g[e] = 0.f;
-    gs[e] = 0.f;
   }
   if (valid) {
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-      g[e] = __ldg(m + col + e) / __ldg(n + col + e);
-      gs[e] = g[e] * s;
-    }
+    for (int e = 0; e < VEC; ++e) g[e] = __ldg(m + col + e) / __ldg(n + col + e);
+    if (HAS_BIAS) bias_raw = VecIO<T, VEC>::raw_param(bias + col);
     const long long row0 = blockIdx.y * rows_per_chunk;
     const long long row1 = min(tokens, row0 + rows_per_chunk);
     long long row = row0 + slot;
     // kBwdRows rows of this thread in flight: their three loads are issued
     // before any is used
     for (; row + (kBwdRows - 1) * kBwdSlots < row1; row += kBwdRows * kBwdSlots) {
-      float a[kBwdRows][VEC], b[kBwdRows][VEC], l[kBwdRows][VEC];
+      Raw ra[kBwdRows], rb[kBwdRows], rl[kBwdRows];
 #pragma unroll
       for (int u = 0; u < kBwdRows; ++u) {
         const long long o = (row + u * kBwdSlots) * d_out + col;
-        VecIO<T, VEC>::load(dy + o, a[u]);
-        VecIO<T, VEC>::load(base + o, b[u]);
-        VecIO<T, VEC>::load(lora + o, l[u]);
+        ra[u] = VecIO<T, VEC>::raw(dy + o);
+        rb[u] = VecIO<T, VEC>::raw(base + o);
+        rl[u] = VecIO<T, VEC>::raw(lora + o);
       }
 #pragma unroll
       for (int u = 0; u < kBwdRows; ++u) {
         const long long o = (row + u * kBwdSlots) * d_out + col;
-        float db[VEC], dl[VEC];
+        float a[VEC], b[VEC], l[VEC], db[VEC], dl[VEC];
+        VecIO<T, VEC>::unpack(ra[u], a);
+        VecIO<T, VEC>::unpack(rb[u], b);
+        VecIO<T, VEC>::unpack(rl[u], l);
+        if (HAS_BIAS) {
+          float bb[VEC];
+          VecIO<T, VEC>::unpack(bias_raw, bb);
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) b[e] -= bb[e];
+        }
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
-          db[e] = g[e] * a[u][e];
-          dl[e] = gs[e] * a[u][e];
-          acc[e] = fmaf(a[u][e], fmaf(s, l[u][e], b[u][e]), acc[e]);
+          db[e] = g[e] * a[e];
+          dl[e] = s * db[e];
+          acc[e] = fmaf(a[e], fmaf(s, l[e], b[e]), acc[e]);
         }
         VecIO<T, VEC>::store(d_base + o, db);
         VecIO<T, VEC>::store(d_lora + o, dl);
@@ -188,10 +238,16 @@ __global__ void __launch_bounds__(kBwdThreads, 2) compose_bwd_kernel(
       VecIO<T, VEC>::load(dy + o0, a0);
       VecIO<T, VEC>::load(base + o0, b0);
       VecIO<T, VEC>::load(lora + o0, l0);
+      if (HAS_BIAS) {
+        float bb[VEC];
+        VecIO<T, VEC>::unpack(bias_raw, bb);
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) b0[e] -= bb[e];
+      }
 #pragma unroll
       for (int e = 0; e < VEC; ++e) {
         db[e] = g[e] * a0[e];
-        dl[e] = gs[e] * a0[e];
+        dl[e] = s * db[e];
         acc[e] = fmaf(a0[e], fmaf(s, l0[e], b0[e]), acc[e]);
       }
       VecIO<T, VEC>::store(d_base + o0, db);

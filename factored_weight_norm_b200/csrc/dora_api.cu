@@ -105,6 +105,19 @@ int make_map(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols) {
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// One compose backward launch; the bias picks the instantiation.
+template <typename T, int VEC>
+void launch_compose_bwd(dim3 grid, cudaStream_t st, const void* dy, const void* base_out, const void* lora_out,
+                        const void* bias, const float* m, const float* n, float s, long long tokens, long long nvec,
+                        long long d_out, void* d_base, void* d_lora, float* part, int* cnt, float* d_m,
+                        long long rows) {
+  auto kernel = bias ? compose_bwd_kernel<T, VEC, true> : compose_bwd_kernel<T, VEC, false>;
+  kernel<<<grid, kBwdThreads, 0, st>>>(static_cast<const T*>(dy), static_cast<const T*>(base_out),
+                                       static_cast<const T*>(lora_out), static_cast<const T*>(bias), m, n, s, tokens,
+                                       nvec, d_out, static_cast<T*>(d_base), static_cast<T*>(d_lora), part, cnt, d_m,
+                                       rows);
+}
+
 // ------------------------------------------------------------ norm planning
 struct TcPlan {
   int m_tiles, n_chunks, chunk_n, kb_main, kb_ext, kb_total;
@@ -441,8 +454,8 @@ int dora_factored_norm(const void* W, const void* A, const void* B, int64_t d_ou
   return launch_error();
 }
 
-int dora_compose_fwd(const void* base_out, const void* lora_out, const float* m, const float* n, float s,
-                     int64_t tokens, int64_t d_out, dora_dtype dt, void* y, void* stream) {
+int dora_compose_fwd(const void* base_out, const void* lora_out, const void* bias, const float* m, const float* n,
+                     float s, int64_t tokens, int64_t d_out, dora_dtype dt, void* y, void* stream) {
   if (dt != DORA_BF16 && dt != DORA_F32) return DORA_ERR_UNSUPPORTED;
   if (tokens < 0 || d_out < 0) return DORA_ERR_INVALID_ARG;
   if (tokens == 0 || d_out == 0) return DORA_OK;
@@ -457,7 +470,7 @@ int dora_compose_fwd(const void* base_out, const void* lora_out, const float* m,
     if (!aligned(base_out, 4) || !aligned(lora_out, 4) || !aligned(y, 4)) return DORA_ERR_UNSUPPORTED;
     vec = (d_out % 4 == 0 && aligned(base_out, 16) && aligned(lora_out, 16) && aligned(y, 16)) ? 4 : 1;
   }
-  if (!aligned(m, 4) || !aligned(n, 4)) return DORA_ERR_UNSUPPORTED;
+  if (!aligned(m, 4) || !aligned(n, 4) || !aligned(bias, dt == DORA_BF16 ? 16 : 4)) return DORA_ERR_UNSUPPORTED;
   DeviceInfo* dev = nullptr;
   if (device_info(&dev)) return DORA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -473,16 +486,18 @@ int dora_compose_fwd(const void* base_out, const void* lora_out, const float* m,
   dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy2));
   if (dt == DORA_BF16)
     compose_fwd_kernel<__nv_bfloat16, 8><<<grid, threads, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(base_out), static_cast<const __nv_bfloat16*>(lora_out), m, n, s, tokens,
-        nvec, d_out, static_cast<__nv_bfloat16*>(y), rows);
+        static_cast<const __nv_bfloat16*>(base_out), static_cast<const __nv_bfloat16*>(lora_out),
+        static_cast<const __nv_bfloat16*>(bias), m, n, s, tokens, nvec, d_out, static_cast<__nv_bfloat16*>(y), rows);
   else if (vec == 4)
     compose_fwd_kernel<float, 4><<<grid, threads, 0, st>>>(static_cast<const float*>(base_out),
-                                                           static_cast<const float*>(lora_out), m, n, s, tokens,
-                                                           nvec, d_out, static_cast<float*>(y), rows);
+                                                           static_cast<const float*>(lora_out),
+                                                           static_cast<const float*>(bias), m, n, s, tokens, nvec,
+                                                           d_out, static_cast<float*>(y), rows);
   else
     compose_fwd_kernel<float, 1><<<grid, threads, 0, st>>>(static_cast<const float*>(base_out),
-                                                           static_cast<const float*>(lora_out), m, n, s, tokens,
-                                                           nvec, d_out, static_cast<float*>(y), rows);
+                                                           static_cast<const float*>(lora_out),
+                                                           static_cast<const float*>(bias), m, n, s, tokens, nvec,
+                                                           d_out, static_cast<float*>(y), rows);
   return launch_error();
 }
 
@@ -492,9 +507,9 @@ size_t dora_compose_bwd_workspace_size(int64_t tokens, int64_t d_out) {
   return align_up(strips * 4, 256) + align_up(static_cast<size_t>(kMaxBwdChunks) * std::max<int64_t>(d_out, 1) * 4, 256);
 }
 
-int dora_compose_bwd(const void* dy, const void* base_out, const void* lora_out, const float* m, const float* n,
-                     float s, int64_t tokens, int64_t d_out, dora_dtype dt, void* d_base, void* d_lora, float* d_m,
-                     void* workspace, size_t workspace_bytes, void* stream) {
+int dora_compose_bwd(const void* dy, const void* base_out, const void* lora_out, const void* bias, const float* m,
+                     const float* n, float s, int64_t tokens, int64_t d_out, dora_dtype dt, void* d_base, void* d_lora,
+                     float* d_m, void* workspace, size_t workspace_bytes, void* stream) {
   if (dt != DORA_BF16 && dt != DORA_F32) return DORA_ERR_UNSUPPORTED;
   if (tokens < 0 || d_out < 0) return DORA_ERR_INVALID_ARG;
   if (d_out == 0) return DORA_OK;
@@ -509,13 +524,14 @@ int dora_compose_bwd(const void* dy, const void* base_out, const void* lora_out,
     vec = 8;
   } else {
     const bool a16 = aligned(dy, 16) && aligned(base_out, 16) && aligned(lora_out, 16) && aligned(d_base, 16) &&
-                     aligned(d_lora, 16);
+                     aligned(d_lora, 16) && aligned(bias, 16);
     if (!aligned(dy, 4) || !aligned(base_out, 4) || !aligned(lora_out, 4) || !aligned(d_base, 4) ||
         !aligned(d_lora, 4))
       return DORA_ERR_UNSUPPORTED;
     vec = (d_out % 4 == 0 && a16) ? 4 : 1;
   }
-  if (!aligned(m, 4) || !aligned(n, 4) || !aligned(d_m, 4)) return DORA_ERR_UNSUPPORTED;
+  if (!aligned(m, 4) || !aligned(n, 4) || !aligned(d_m, 4) || !aligned(bias, dt == DORA_BF16 ? 16 : 4))
+    return DORA_ERR_UNSUPPORTED;
   const size_t need = dora_compose_bwd_workspace_size(tokens, d_out);
   if (!workspace || workspace_bytes < need) return DORA_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return DORA_ERR_UNSUPPORTED;
@@ -529,11 +545,11 @@ int dora_compose_bwd(const void* dy, const void* base_out, const void* lora_out,
   if (strips > INT32_MAX) return DORA_ERR_UNSUPPORTED;
   int occ = 1;
   if (dt == DORA_BF16)
-    occ = ctas_per_sm(compose_bwd_kernel<__nv_bfloat16, 8>, kBwdThreads);
+    occ = ctas_per_sm(compose_bwd_kernel<__nv_bfloat16, 8, false>, kBwdThreads);
   else if (vec == 4)
-    occ = ctas_per_sm(compose_bwd_kernel<float, 4>, kBwdThreads);
+    occ = ctas_per_sm(compose_bwd_kernel<float, 4, false>, kBwdThreads);
   else
-    occ = ctas_per_sm(compose_bwd_kernel<float, 1>, kBwdThreads);
+    occ = ctas_per_sm(compose_bwd_kernel<float, 1, false>, kBwdThreads);
   // about two waves of resident CTAs
   const long long chunks = std::max<long long>(
       1, std::min<long long>({2LL * dev->num_sms * occ / strips, kMaxBwdChunks, cdiv(tokens, kBwdSlots)}));
@@ -546,18 +562,14 @@ int dora_compose_bwd(const void* dy, const void* base_out, const void* lora_out,
   if (cudaMemsetAsync(cnt, 0, static_cast<size_t>(strips) * 4, st) != cudaSuccess) return DORA_ERR_CUDA;
   dim3 grid(static_cast<unsigned>(strips), static_cast<unsigned>(chunks2));
   if (dt == DORA_BF16)
-    compose_bwd_kernel<__nv_bfloat16, 8><<<grid, kBwdThreads, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(dy), static_cast<const __nv_bfloat16*>(base_out),
-        static_cast<const __nv_bfloat16*>(lora_out), m, n, s, tokens, nvec, d_out,
-        static_cast<__nv_bfloat16*>(d_base), static_cast<__nv_bfloat16*>(d_lora), part, cnt, d_m, rows);
+    launch_compose_bwd<__nv_bfloat16, 8>(grid, st, dy, base_out, lora_out, bias, m, n, s, tokens, nvec, d_out, d_base,
+                                         d_lora, part, cnt, d_m, rows);
   else if (vec == 4)
-    compose_bwd_kernel<float, 4><<<grid, kBwdThreads, 0, st>>>(
-        static_cast<const float*>(dy), static_cast<const float*>(base_out), static_cast<const float*>(lora_out), m, n,
-        s, tokens, nvec, d_out, static_cast<float*>(d_base), static_cast<float*>(d_lora), part, cnt, d_m, rows);
+    launch_compose_bwd<float, 4>(grid, st, dy, base_out, lora_out, bias, m, n, s, tokens, nvec, d_out, d_base, d_lora,
+                                part, cnt, d_m, rows);
   else
-    compose_bwd_kernel<float, 1><<<grid, kBwdThreads, 0, st>>>(
-        static_cast<const float*>(dy), static_cast<const float*>(base_out), static_cast<const float*>(lora_out), m, n,
-        s, tokens, nvec, d_out, static_cast<float*>(d_base), static_cast<float*>(d_lora), part, cnt, d_m, rows);
+    launch_compose_bwd<float, 1>(grid, st, dy, base_out, lora_out, bias, m, n, s, tokens, nvec, d_out, d_base, d_lora,
+                                part, cnt, d_m, rows);
   return launch_error();
 }
 
@@ -668,9 +680,9 @@ int noalloc_scratch(unsigned char** out) {
 }  // namespace
 }  // namespace dora
 
-extern "C" int dora_compose_bwd_noalloc(const void* dy, const void* base_out, const void* lora_out, const float* m,
-                                        const float* n, float s, int64_t tokens, int64_t d_out, dora_dtype dt,
-                                        void* d_base, void* d_lora, float* d_m, void* stream) {
+extern "C" int dora_compose_bwd_noalloc(const void* dy, const void* base_out, const void* lora_out, const void* bias,
+                                        const float* m, const float* n, float s, int64_t tokens, int64_t d_out,
+                                        dora_dtype dt, void* d_base, void* d_lora, float* d_m, void* stream) {
   if (dt != DORA_BF16 && dt != DORA_F32) return DORA_ERR_UNSUPPORTED;
   if (tokens < 0 || d_out < 0) return DORA_ERR_INVALID_ARG;
   if (d_out > DORA_NOALLOC_MAX_D_OUT) return DORA_ERR_UNSUPPORTED;
@@ -686,13 +698,14 @@ extern "C" int dora_compose_bwd_noalloc(const void* dy, const void* base_out, co
     vec = 8;
   } else {
     const bool a16 = aligned(dy, 16) && aligned(base_out, 16) && aligned(lora_out, 16) && aligned(d_base, 16) &&
-                     aligned(d_lora, 16);
+                     aligned(d_lora, 16) && aligned(bias, 16);
     if (!aligned(dy, 4) || !aligned(base_out, 4) || !aligned(lora_out, 4) || !aligned(d_base, 4) ||
         !aligned(d_lora, 4))
       return DORA_ERR_UNSUPPORTED;
     vec = (d_out % 4 == 0 && a16) ? 4 : 1;
   }
-  if (!aligned(m, 4) || !aligned(n, 4) || !aligned(d_m, 4)) return DORA_ERR_UNSUPPORTED;
+  if (!aligned(m, 4) || !aligned(n, 4) || !aligned(d_m, 4) || !aligned(bias, dt == DORA_BF16 ? 16 : 4))
+    return DORA_ERR_UNSUPPORTED;
   DeviceInfo* dev = nullptr;
   if (device_info(&dev)) return DORA_ERR_CUDA;
   unsigned char* scratch = nullptr;
@@ -704,11 +717,11 @@ extern "C" int dora_compose_bwd_noalloc(const void* dy, const void* base_out, co
   const long long strips = cdiv(nvec, kBwdVecs);
   int occ = 1;
   if (dt == DORA_BF16)
-    occ = ctas_per_sm(compose_bwd_kernel<__nv_bfloat16, 8>, kBwdThreads);
+    occ = ctas_per_sm(compose_bwd_kernel<__nv_bfloat16, 8, false>, kBwdThreads);
   else if (vec == 4)
-    occ = ctas_per_sm(compose_bwd_kernel<float, 4>, kBwdThreads);
+    occ = ctas_per_sm(compose_bwd_kernel<float, 4, false>, kBwdThreads);
   else
-    occ = ctas_per_sm(compose_bwd_kernel<float, 1>, kBwdThreads);
+    occ = ctas_per_sm(compose_bwd_kernel<float, 1, false>, kBwdThreads);
   const long long chunks = pick_chunks(strips, static_cast<long long>(dev->num_sms) * occ,
                                        std::min<long long>(kNoallocChunks, cdiv(tokens, kBwdSlots)));
   const long long rows = cdiv(tokens, chunks);
@@ -719,17 +732,13 @@ extern "C" int dora_compose_bwd_noalloc(const void* dy, const void* base_out, co
   if (cudaMemsetAsync(cnt, 0, static_cast<size_t>(strips) * 4, st) != cudaSuccess) return DORA_ERR_CUDA;
   dim3 grid(static_cast<unsigned>(strips), static_cast<unsigned>(chunks2));
   if (dt == DORA_BF16)
-    compose_bwd_kernel<__nv_bfloat16, 8><<<grid, kBwdThreads, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(dy), static_cast<const __nv_bfloat16*>(base_out),
-        static_cast<const __nv_bfloat16*>(lora_out), m, n, s, tokens, nvec, d_out,
-        static_cast<__nv_bfloat16*>(d_base), static_cast<__nv_bfloat16*>(d_lora), part, cnt, d_m, rows);
+    launch_compose_bwd<__nv_bfloat16, 8>(grid, st, dy, base_out, lora_out, bias, m, n, s, tokens, nvec, d_out, d_base,
+                                         d_lora, part, cnt, d_m, rows);
   else if (vec == 4)
-    compose_bwd_kernel<float, 4><<<grid, kBwdThreads, 0, st>>>(
-        static_cast<const float*>(dy), static_cast<const float*>(base_out), static_cast<const float*>(lora_out), m, n,
-        s, tokens, nvec, d_out, static_cast<float*>(d_base), static_cast<float*>(d_lora), part, cnt, d_m, rows);
+    launch_compose_bwd<float, 4>(grid, st, dy, base_out, lora_out, bias, m, n, s, tokens, nvec, d_out, d_base, d_lora,
+                                part, cnt, d_m, rows);
   else
-    compose_bwd_kernel<float, 1><<<grid, kBwdThreads, 0, st>>>(
-        static_cast<const float*>(dy), static_cast<const float*>(base_out), static_cast<const float*>(lora_out), m, n,
-        s, tokens, nvec, d_out, static_cast<float*>(d_base), static_cast<float*>(d_lora), part, cnt, d_m, rows);
+    launch_compose_bwd<float, 1>(grid, st, dy, base_out, lora_out, bias, m, n, s, tokens, nvec, d_out, d_base, d_lora,
+                                part, cnt, d_m, rows);
   return launch_error();
 }

@@ -48,17 +48,17 @@ SIGNATURES = {
     ),
     "dora_compose_fwd": (
         ctypes.c_int,
-        [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _f32, _i64, _i64, ctypes.c_int, _c_void_p, _c_void_p],
+        [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _f32, _i64, _i64, ctypes.c_int, _c_void_p, _c_void_p],
     ),
     "dora_compose_bwd_workspace_size": (_size, [_i64, _i64]),
     "dora_compose_bwd": (
         ctypes.c_int,
-        [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _f32, _i64, _i64, ctypes.c_int,
+        [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _f32, _i64, _i64, ctypes.c_int,
          _c_void_p, _c_void_p, _c_void_p, _c_void_p, _size, _c_void_p],
     ),
     "dora_compose_bwd_noalloc": (
         ctypes.c_int,
-        [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _f32, _i64, _i64, ctypes.c_int,
+        [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _f32, _i64, _i64, ctypes.c_int,
          _c_void_p, _c_void_p, _c_void_p, _c_void_p],
     ),
     "dora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -222,18 +222,32 @@ def dora_factored_norm_batched(modules, n_outs=None, workspace=None, stream=None
     return n_outs
 
 
-def dora_compose_fwd(base_out, lora_out, m, n, s: float, y=None, stream=None):
-    """y = (m / n) * (base_out + s * lora_out), single fused pass."""
+def _check_bias(bias, base_out, name):
+    if bias is None:
+        return
+    _dense_cuda(bias)
+    if bias.shape != (base_out.shape[1],):
+        raise ValueError(f"bias must have shape (d_out,) in {name}")
+    if bias.dtype != base_out.dtype:
+        raise TypeError(f"bias must have the activations' dtype in {name}")
+
+
+def dora_compose_fwd(base_out, lora_out, m, n, s: float, y=None, stream=None, bias=None):
+    """y = b + (m / n) * ((base_out - b) + s * lora_out), single fused pass.
+
+    base_out is the base layer's output including its bias b (``bias``,
+    ``None`` for a layer without one)."""
     _dense_cuda(base_out, lora_out, m, n, y)
     tokens, d_out = base_out.shape
     if lora_out.shape != base_out.shape or m.shape != (d_out,) or n.shape != (d_out,):
         raise ValueError("shape mismatch in dora_compose_fwd")
     if m.dtype != torch.float32 or n.dtype != torch.float32:
         raise TypeError("m and n must be fp32")
+    _check_bias(bias, base_out, "dora_compose_fwd")
     if y is None:
         y = torch.empty_like(base_out)
     st = lib().dora_compose_fwd(
-        _ptr(base_out), _ptr(lora_out), _ptr(m), _ptr(n), float(s), tokens, d_out, _dt(base_out), _ptr(y),
+        _ptr(base_out), _ptr(lora_out), _ptr(bias), _ptr(m), _ptr(n), float(s), tokens, d_out, _dt(base_out), _ptr(y),
         _stream(stream),
     )
     _check(st, "dora_compose_fwd")
@@ -241,14 +255,15 @@ def dora_compose_fwd(base_out, lora_out, m, n, s: float, y=None, stream=None):
 
 
 def dora_compose_bwd(dy, base_out, lora_out, m, n, s: float, d_base=None, d_lora=None, d_m=None, workspace=None,
-                     stream=None):
-    """(d_base, d_lora, d_m) of the compose with n held constant."""
+                     stream=None, bias=None):
+    """(d_base, d_lora, d_m) of the compose with n held constant and the bias frozen."""
     _dense_cuda(dy, base_out, lora_out, m, n, d_base, d_lora, d_m, workspace)
     tokens, d_out = base_out.shape
     if dy.shape != base_out.shape or lora_out.shape != base_out.shape:
         raise ValueError("shape mismatch in dora_compose_bwd")
     if m.dtype != torch.float32 or n.dtype != torch.float32:
         raise TypeError("m and n must be fp32")
+    _check_bias(bias, base_out, "dora_compose_bwd")
     if d_base is None:
         d_base = torch.empty_like(base_out)
     if d_lora is None:
@@ -259,9 +274,29 @@ def dora_compose_bwd(dy, base_out, lora_out, m, n, s: float, d_base=None, d_lora
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=base_out.device)
     st = lib().dora_compose_bwd(
-        _ptr(dy), _ptr(base_out), _ptr(lora_out), _ptr(m), _ptr(n), float(s), tokens, d_out, _dt(base_out),
-        _ptr(d_base), _ptr(d_lora), _ptr(d_m), _ptr(workspace), workspace.numel() * workspace.element_size(),
-        _stream(stream),
+        _ptr(dy), _ptr(base_out), _ptr(lora_out), _ptr(bias), _ptr(m), _ptr(n), float(s), tokens, d_out,
+        _dt(base_out), _ptr(d_base), _ptr(d_lora), _ptr(d_m), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream),
     )
     _check(st, "dora_compose_bwd")
+    return d_base, d_lora, d_m
+
+
+def dora_compose_bwd_noalloc(dy, base_out, lora_out, m, n, s: float, d_base, d_lora, d_m, stream=None, bias=None):
+    """dora_compose_bwd into caller-provided outputs, with the library's own
+    scratch instead of a workspace (nothing is allocated)."""
+    _dense_cuda(dy, base_out, lora_out, m, n, d_base, d_lora, d_m)
+    tokens, d_out = base_out.shape
+    if dy.shape != base_out.shape or lora_out.shape != base_out.shape:
+        raise ValueError("shape mismatch in dora_compose_bwd_noalloc")
+    if d_base.shape != base_out.shape or d_lora.shape != base_out.shape or d_m.shape != (d_out,):
+        raise ValueError("output shape mismatch in dora_compose_bwd_noalloc")
+    if m.dtype != torch.float32 or n.dtype != torch.float32 or d_m.dtype != torch.float32:
+        raise TypeError("m, n and d_m must be fp32")
+    _check_bias(bias, base_out, "dora_compose_bwd_noalloc")
+    st = lib().dora_compose_bwd_noalloc(
+        _ptr(dy), _ptr(base_out), _ptr(lora_out), _ptr(bias), _ptr(m), _ptr(n), float(s), tokens, d_out,
+        _dt(base_out), _ptr(d_base), _ptr(d_lora), _ptr(d_m), _stream(stream),
+    )
+    _check(st, "dora_compose_bwd_noalloc")
     return d_base, d_lora, d_m
