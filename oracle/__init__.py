@@ -11,6 +11,7 @@ from .dora_oracle import (  # noqa: F401
     compose_backward_columns,
     compose_forward,
     dense_adapted_weight,
+    linear_forward,
     magnitude_scale,
     row_norm,
     row_norm_rows,

@@ -77,6 +77,7 @@ __all__ = [
     "compose_forward",
     "compose_backward",
     "compose_backward_columns",
+    "linear_forward",
 ]
 
 
@@ -177,3 +178,23 @@ def compose_backward_columns(dy, base, lora, m, n, s, cols, bias=None) -> np.nda
     b_c = None if bias is None else _f64(bias)[cols]
     _, _, d_m = compose_backward(dy_c, base_c, lora_c, _f64(m)[cols], _f64(n)[cols], s, bias=b_c)
     return d_m
+
+
+def linear_forward(x, W, A, B, m, n, s, bias=None, cols=None) -> np.ndarray:
+    """The adapted layer's output ``y = b + (m / n) * (x W'^T)``, ``W' = W + s B A``.
+
+    DoRA summary page, Method: the adapted weight is the magnitude times the
+    per-channel normalised direction ``W' / ||W'||`` (here with the given ``n``
+    standing for ``||W'_i||``); the layer applies it to ``x`` ``[tokens, d_in]``
+    and adds the frozen bias ``b`` (``None``: no bias).  Scaling DoRA,
+    Abstract: this is the output the fused composition produces.  ``cols``
+    restricts the result to those output channels (``W'`` is formed densely
+    for them only); ``None`` means all.
+    """
+    x, W, A, B = _f64(x), _f64(W), _f64(A), _f64(B)
+    d_out = W.shape[0]
+    cols = np.arange(d_out) if cols is None else np.asarray(cols, dtype=np.int64)
+    Wp = dense_adapted_weight(W[cols], A, B[cols], s)
+    g = magnitude_scale(_f64(m)[cols], _f64(n)[cols])
+    b = _bias(bias, d_out)[cols]
+    return b[None, :] + g[None, :] * (x @ Wp.T)

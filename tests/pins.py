@@ -23,6 +23,10 @@ Method):
                      the forward definition with n held constant;
 * hand-worked      - small integer cases with exact answers worked by hand,
                      stored in tests/golden/hand_cases.json;
+* layer            - the adapted layer (dense W' = W + sBA applied to x,
+                     rescaled per output channel, plus b) equals pure-Python
+                     loops on tiny shapes and the separately pinned compose
+                     form fed base = x W^T + b and lora = (x A^T) B^T;
 * bias             - the compose form with a bias (base = x W^T + b) equals
                      the adapted layer itself, x (diag(m / n) (W + sBA))^T + b
                      with n from numpy.linalg.norm, and its d_m equals
@@ -286,6 +290,40 @@ def pin_bias_layer(compose_forward, compose_backward, seed=6):
         d_base0, d_lora0, _ = compose_backward(dy, base, lora, m, n, s)
         assert np.array_equal(d_base, d_base0) and np.array_equal(d_lora, d_lora0)
         assert np.max(np.abs(d_base - (m / n)[None, :] * dy)) < 1e-15 * (1 + np.max(np.abs(d_base)))
+
+
+# ----------------------------------------------------------------- layer
+def brute_layer(x, W, A, B, m, n, s, b):
+    T, d_in, d_out, r = len(x), len(W[0]), len(W), len(A)
+    y = [[0.0] * d_out for _ in range(T)]
+    for i in range(d_out):
+        row = [W[i][k] + s * sum(B[i][j] * A[j][k] for j in range(r)) for k in range(d_in)]
+        for t in range(T):
+            y[t][i] = b[i] + (m[i] / n[i]) * sum(x[t][k] * row[k] for k in range(d_in))
+    return y
+
+
+def pin_layer(linear_forward, compose_forward, seed=7):
+    rng = np.random.default_rng(seed)
+    for T, d_in, d_out, r in ((1, 1, 1, 1), (3, 5, 4, 2), (6, 9, 7, 3)):
+        x = rng.standard_normal((T, d_in))
+        W, A, B = tiny_case(rng, d_out, d_in, r)
+        b = rng.standard_normal(d_out)
+        n = rng.uniform(0.5, 2.0, d_out)
+        m = n * rng.uniform(0.8, 1.2, d_out)
+        for s in (0.0, 0.75, -1.5):
+            ref = np.array(brute_layer(x.tolist(), W.tolist(), A.tolist(), B.tolist(), m.tolist(), n.tolist(), s,
+                                       b.tolist()))
+            y = linear_forward(x, W, A, B, m, n, s, bias=b)
+            assert np.shape(y) == (T, d_out)
+            assert np.max(np.abs(y - ref)) <= 1e-12 * (1 + np.max(np.abs(ref)))
+            y2 = compose_forward(x @ W.T + b[None, :], (x @ A.T) @ B.T, m, n, s, bias=b)
+            assert np.max(np.abs(y - y2)) <= 1e-12 * (1 + np.max(np.abs(ref)))
+            cols = [d_out - 1, 0]
+            assert np.max(np.abs(linear_forward(x, W, A, B, m, n, s, bias=b, cols=cols) - ref[:, cols])) <= 1e-12 * (
+                1 + np.max(np.abs(ref)))
+            y0 = linear_forward(x, W, A, B, m, n, s)
+            assert np.max(np.abs(y0 - (ref - b[None, :]))) <= 1e-12 * (1 + np.max(np.abs(ref)))
 
 
 # ------------------------------------------------------------ hand-worked

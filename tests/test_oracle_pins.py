@@ -31,6 +31,46 @@ def test_finite_differences():
     pins.pin_finite_differences(oracle.compose_forward, oracle.compose_backward)
 
 
+def test_layer():
+    pins.pin_layer(oracle.linear_forward, oracle.compose_forward)
+
+
+def _l_g_on_rows(x, W, A, B, m, n, s, bias=None, cols=None):
+    y = oracle.linear_forward(x, W, A, B, np.ones(len(m)), np.ones(len(n)), s, bias=bias, cols=cols)
+    b = 0.0 if bias is None else np.asarray(bias, float)[None, :]
+    if cols is not None:
+        b = b if bias is None else np.asarray(bias, float)[cols][None, :]
+    g = np.asarray(m, float) / np.asarray(n, float)
+    T = y.shape[0]
+    return b + g[:T, None] * (y - b) if T <= len(g) else y
+
+
+def _l_no_s(x, W, A, B, m, n, s, bias=None, cols=None):
+    return oracle.linear_forward(x, W, A, B, m, n, 1.0, bias=bias, cols=cols)
+
+
+def _l_transposed_A(x, W, A, B, m, n, s, bias=None, cols=None):
+    A = np.asarray(A, float)
+    return oracle.linear_forward(x, W, A[::-1], B, m, n, s, bias=bias, cols=cols)
+
+
+def _l_bias_scaled(x, W, A, B, m, n, s, bias=None, cols=None):
+    y = oracle.linear_forward(x, W, A, B, m, n, s, cols=cols)
+    if bias is None:
+        return y
+    b = np.asarray(bias, float)
+    b = b if cols is None else b[cols]
+    g = np.asarray(m, float) / np.asarray(n, float)
+    g = g if cols is None else g[cols]
+    return y + (g * b)[None, :]
+
+
+@pytest.mark.parametrize("mutant", [_l_g_on_rows, _l_no_s, _l_transposed_A, _l_bias_scaled], ids=lambda f: f.__name__)
+def test_layer_mutant_is_caught(mutant):
+    with pytest.raises((AssertionError, ValueError)):
+        pins.pin_layer(mutant, oracle.compose_forward)
+
+
 def test_bias_layer():
     pins.pin_bias_layer(oracle.compose_forward, oracle.compose_backward)
 
