@@ -16,6 +16,7 @@
 
 #include "../../include/dora.h"
 #include "compose.cuh"
+#include "linear_tc.cuh"
 #include "norm_simt.cuh"
 #include "norm_tc.cuh"
 #include "norm_batched.cuh"
@@ -30,6 +31,14 @@ __device__ int g_status = 0;
 namespace {
 
 constexpr long long kWaitLimitCycles = 2000000000LL;  // ~1 s at B200 clocks
+
+// linear_pair_kernel: as many 32 KB stages as fit, at most kLinStagesMax
+int linear_pair_stages(int smem_optin) {
+  return static_cast<int>(std::min<size_t>(kLinStagesMax, (smem_optin - 1024 - kLinBarrierBytes) / kPairStageBytes));
+}
+size_t linear_pair_smem(int smem_optin) {
+  return static_cast<size_t>(linear_pair_stages(smem_optin)) * kPairStageBytes + 1024 + kLinBarrierBytes;
+}
 constexpr int kMaxGrid = 1024;                         // bound on the persistent grid
 constexpr int kMaxGramSplits = 32;
 constexpr int kMaxBwdChunks = 64;
@@ -44,6 +53,7 @@ struct DeviceInfo {
   int num_sms = 0;
   int smem_optin = 0;
   int* status = nullptr;
+  int pair_clusters = 0;  // co-resident 2-CTA clusters of linear_pair_kernel
 };
 
 std::mutex g_mu;
@@ -76,6 +86,26 @@ int device_info(DeviceInfo** out) {
         cudaFuncSetAttribute(gram_batched_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin) !=
             cudaSuccess)
       return DORA_ERR_CUDA;
+    if (cudaFuncSetAttribute(linear_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(linear_pair_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess)
+      return DORA_ERR_CUDA;
+    {
+      cudaLaunchConfig_t occ{};
+      cudaLaunchAttribute cl[1];
+      cl[0].id = cudaLaunchAttributeClusterDimension;
+      cl[0].val.clusterDim.x = 2;
+      cl[0].val.clusterDim.y = 1;
+      cl[0].val.clusterDim.z = 1;
+      occ.gridDim = dim3(2 * (d.num_sms / 2));
+      occ.blockDim = dim3(kLinThreads);
+      occ.dynamicSmemBytes = linear_pair_smem(d.smem_optin);
+      occ.attrs = cl;
+      occ.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&d.pair_clusters, linear_pair_kernel, &occ) != cudaSuccess ||
+          d.pair_clusters < 1)
+        return DORA_ERR_CUDA;
+    }
     if (!g_encode) {
       void* fn = nullptr;
       cudaDriverEntryPointQueryResult q;
@@ -92,10 +122,10 @@ int device_info(DeviceInfo** out) {
 
 // 2-D bf16 tensor map over a row-major [rows, cols] matrix, 64 x 128 boxes,
 // 128-byte swizzle, zero fill outside the matrix.
-int make_map(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols) {
+int make_map(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows = kBoxRows) {
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(kBoxRows)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
                               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -639,6 +669,107 @@ int dora_num_sms(void) {
   DeviceInfo* dev = nullptr;
   if (device_info(&dev)) return 0;
   return dev->num_sms;
+}
+
+
+size_t dora_fused_linear_fwd_workspace_size(int64_t tokens, int64_t r) {
+  if (tokens < 0 || r < 0) return 0;
+  return std::max<size_t>(256, align_up(static_cast<size_t>(tokens) * static_cast<size_t>(r) * 2, 256));
+}
+
+int dora_fused_linear_fwd(const void* x, const void* W, const void* A, const void* B, const void* bias, const float* m,
+                          const float* n, float s, int64_t tokens, int64_t d_in, int64_t d_out, int64_t r,
+                          dora_dtype dt, void* y, void* workspace, size_t workspace_bytes, void* stream) {
+  if (dt != DORA_BF16) return DORA_ERR_UNSUPPORTED;
+  if (tokens < 0 || d_in < 0 || d_out < 0 || r < 0) return DORA_ERR_INVALID_ARG;
+  if (tokens == 0 || d_out == 0) return DORA_OK;
+  if (d_in == 0) return DORA_ERR_UNSUPPORTED;
+  if (tokens > INT32_MAX / 2 || d_in > INT32_MAX / 2 || d_out > INT32_MAX / 2 || r > INT32_MAX / 2)
+    return DORA_ERR_UNSUPPORTED;
+  if (!x || !W || !m || !n || !y || (r > 0 && (!A || !B))) return DORA_ERR_INVALID_ARG;
+  if (d_in % 8 != 0 || d_out % 8 != 0 || r % 8 != 0) return DORA_ERR_UNSUPPORTED;
+  if (!aligned(x, 16) || !aligned(W, 16) || !aligned(A, 16) || !aligned(B, 16) || !aligned(y, 16) ||
+      !aligned(bias, 2) || !aligned(m, 4) || !aligned(n, 4))
+    return DORA_ERR_UNSUPPORTED;
+  if (cdiv(tokens, kPairBM) * cdiv(d_out, kPairBN) > INT32_MAX) return DORA_ERR_UNSUPPORTED;
+  const size_t need = dora_fused_linear_fwd_workspace_size(tokens, r);
+  if (r > 0 && (!workspace || workspace_bytes < need)) return DORA_ERR_WORKSPACE;
+  if (r > 0 && !aligned(workspace, 256)) return DORA_ERR_UNSUPPORTED;
+  DeviceInfo* dev = nullptr;
+  if (device_info(&dev)) return DORA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  __nv_bfloat16* P = static_cast<__nv_bfloat16*>(workspace);
+
+  CUtensorMap tmX, tmW, tmA, tmP, tmB;
+  if (make_map(&tmX, x, tokens, d_in) || make_map(&tmW, W, d_out, d_in)) return DORA_ERR_CUDA;
+  if (r > 0 && (make_map(&tmA, A, r, d_in) || make_map(&tmP, P, tokens, r) || make_map(&tmB, B, d_out, r)))
+    return DORA_ERR_CUDA;
+  const int kb_main = static_cast<int>(cdiv(d_in, kLinBK));
+  const int stages = linear_pair_stages(dev->smem_optin);
+  if (stages < 2) return DORA_ERR_UNSUPPORTED;
+  const long long tiles_m2 = cdiv(tokens, kPairBM);
+
+  cudaLaunchAttribute attrs[2];
+  attrs[0].id = cudaLaunchAttributeClusterDimension;
+  attrs[0].val.clusterDim.x = 2;
+  attrs[0].val.clusterDim.y = 1;
+  attrs[0].val.clusterDim.z = 1;
+  attrs[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[1].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.stream = st;
+  cfg.attrs = attrs;
+  cfg.blockDim = dim3(kLinThreads);
+  cfg.dynamicSmemBytes = linear_pair_smem(dev->smem_optin);
+  auto pairs_for = [&](long long tiles) {
+    return static_cast<unsigned>(2 * std::min<long long>(dev->pair_clusters, tiles));
+  };
+
+  // 1) P = bf16(s * x A^T) into the workspace
+  if (r > 0) {
+    LinearArgs pa{};
+    pa.M = static_cast<int>(tokens);
+    pa.N = static_cast<int>(r);
+    pa.kb_main = pa.kb_total = kb_main;
+    pa.tiles_m = static_cast<int>(tiles_m2);
+    pa.tiles_n = static_cast<int>(cdiv(r, kPairBN));
+    pa.stages = stages;
+    pa.stage_bytes = kPairStageBytes;
+    pa.alpha = s;
+    pa.out = P;
+    pa.ldo = r;
+    pa.wait_limit = kWaitLimitCycles;
+    pa.status = dev->status;
+    cfg.numAttrs = 1;  // cluster shape only: ordered after everything before it on the stream
+    cfg.gridDim = dim3(pairs_for(static_cast<long long>(pa.tiles_m) * pa.tiles_n));
+    if (cudaLaunchKernelEx(&cfg, linear_pair_kernel, tmX, tmA, tmX, tmA, pa) != cudaSuccess) return DORA_ERR_CUDA;
+  }
+
+  // 2) y = bf16(g * [x | P] [W | B]^T + b), dependent on 1) only for the extension blocks
+  LinearArgs la{};
+  la.M = static_cast<int>(tokens);
+  la.N = static_cast<int>(d_out);
+  la.kb_main = kb_main;
+  la.kb_total = kb_main + static_cast<int>(cdiv(r, kLinBK));
+  la.tiles_m = static_cast<int>(tiles_m2);
+  la.tiles_n = static_cast<int>(cdiv(d_out, kPairBN));
+  la.stages = stages;
+  la.stage_bytes = kPairStageBytes;
+  la.alpha = 1.f;
+  la.m = m;
+  la.n = n;
+  la.bias = static_cast<const __nv_bfloat16*>(bias);
+  la.out = static_cast<__nv_bfloat16*>(y);
+  la.ldo = d_out;
+  la.ext_waits = r > 0 ? 1 : 0;
+  la.wait_limit = kWaitLimitCycles;
+  la.status = dev->status;
+  cfg.numAttrs = r > 0 ? 2 : 1;
+  cfg.gridDim = dim3(pairs_for(static_cast<long long>(la.tiles_m) * la.tiles_n));
+  const CUtensorMap& tmA2 = r > 0 ? tmP : tmX;
+  const CUtensorMap& tmB2 = r > 0 ? tmB : tmW;
+  if (cudaLaunchKernelEx(&cfg, linear_pair_kernel, tmX, tmW, tmA2, tmB2, la) != cudaSuccess) return DORA_ERR_CUDA;
+  return launch_error();
 }
 
 }  // extern "C"

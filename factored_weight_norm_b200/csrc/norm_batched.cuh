@@ -31,12 +31,6 @@ struct alignas(64) BatchDesc {
   float two_s, half_s;
 };
 
-// Two floats as packed bf16 (round to nearest even), low half first.
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-
 // (module, tile) of a work list entry
 struct BatchItem {
   int prob, tile;

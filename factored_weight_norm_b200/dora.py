@@ -67,6 +67,12 @@ SIGNATURES = {
     "dora_selftest_timeout": (ctypes.c_int, [_i64, _c_void_p]),
     "dora_factored_norm_batched_workspace_size": (_size, [_problems_p, ctypes.c_int, ctypes.c_int]),
     "dora_factored_norm_batched": (ctypes.c_int, [_problems_p, ctypes.c_int, ctypes.c_int, _c_void_p, _size, _c_void_p]),
+    "dora_fused_linear_fwd_workspace_size": (_size, [_i64, _i64]),
+    "dora_fused_linear_fwd": (
+        ctypes.c_int,
+        [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _f32, _i64, _i64, _i64, _i64,
+         ctypes.c_int, _c_void_p, _c_void_p, _size, _c_void_p],
+    ),
 }
 
 _lib = None
@@ -300,3 +306,36 @@ def dora_compose_bwd_noalloc(dy, base_out, lora_out, m, n, s: float, d_base, d_l
     )
     _check(st, "dora_compose_bwd_noalloc")
     return d_base, d_lora, d_m
+
+
+def dora_fused_linear_fwd_workspace_size(tokens: int, r: int) -> int:
+    return int(lib().dora_fused_linear_fwd_workspace_size(tokens, r))
+
+
+def dora_fused_linear_fwd(x, W, A, B, m, n, s: float, bias=None, y=None, workspace=None, stream=None):
+    """y = b + (m / n) * (x W^T + s * (x A^T) B^T), the compose fused into the GEMMs (bf16)."""
+    _dense_cuda(x, W, A, B, m, n, bias, y, workspace)
+    T, d_in = x.shape
+    d_out, r = W.shape[0], A.shape[0]
+    if W.shape != (d_out, d_in) or A.shape != (r, d_in) or B.shape != (d_out, r):
+        raise ValueError("shape mismatch in dora_fused_linear_fwd")
+    if m.shape != (d_out,) or n.shape != (d_out,):
+        raise ValueError("m and n must have shape (d_out,)")
+    if m.dtype != torch.float32 or n.dtype != torch.float32:
+        raise TypeError("m and n must be fp32")
+    for t in (x, W, A, B):
+        if t.dtype != torch.bfloat16:
+            raise TypeError("x, W, A and B must be bf16")
+    if bias is not None and (bias.shape != (d_out,) or bias.dtype != torch.bfloat16):
+        raise ValueError("bias must be bf16 of shape (d_out,)")
+    if y is None:
+        y = torch.empty(T, d_out, dtype=torch.bfloat16, device=x.device)
+    need = dora_fused_linear_fwd_workspace_size(T, r)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    st = lib().dora_fused_linear_fwd(
+        _ptr(x), _ptr(W), _ptr(A), _ptr(B), _ptr(bias), _ptr(m), _ptr(n), float(s), T, d_in, d_out, r, DORA_BF16,
+        _ptr(y), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream),
+    )
+    _check(st, "dora_fused_linear_fwd")
+    return y

@@ -182,6 +182,38 @@ DORA_API int dora_compose_bwd_noalloc(const void* dy, const void* base_out, cons
                                       const float* m, const float* n, float s, int64_t tokens, int64_t d_out,
                                       dora_dtype dt, void* d_base, void* d_lora, float* d_m, void* stream);
 
+/* Bytes of workspace dora_fused_linear_fwd needs: the [tokens, r] bf16
+ * intermediate P = s * x A^T (at least 256). */
+DORA_API size_t dora_fused_linear_fwd_workspace_size(int64_t tokens, int64_t r);
+
+/* The DoRA linear forward with the compose fused into the GEMMs that produce
+ * its inputs (Scaling DoRA, Abstract: the composition collapsed into one pass
+ * over the activations; here the pass is the GEMM epilogue itself, so the
+ * base and LoRA outputs are never written to memory):
+ *
+ *   y = b + g * (x W^T + s * (x A^T) B^T),   g = m / n   per output channel
+ *
+ * computed as P = bf16(s * x A^T) (one tcgen05 GEMM into the workspace), then
+ * y = bf16(g * [x | P] [W | B]^T + b) (one tcgen05 GEMM whose K runs over d_in
+ * and then r; fp32 accumulation, g and b applied in fp32, one rounding).
+ * This equals dora_compose_fwd applied to base = x W^T + b and
+ * lora = (x A^T) B^T, except that P is rounded to bf16 once, as a framework's
+ * LoRA path rounds x A^T.
+ *
+ * x: [tokens, d_in]; W: [d_out, d_in]; A: [r, d_in]; B: [d_out, r]; y:
+ * [tokens, d_out]; all bf16, row-major, 16-byte aligned; d_in, d_out, r
+ * multiples of 8; d_in > 0.  bias: bf16 [d_out] or NULL.  m, n: fp32
+ * [d_out] (n from dora_factored_norm).  r = 0 gives y = b + g * x W^T (no
+ * workspace needed).  workspace: device buffer of at least
+ * dora_fused_linear_fwd_workspace_size(tokens, r) bytes, 256-byte aligned,
+ * contents ignored on entry.  Only dt = DORA_BF16 is accepted
+ * (DORA_ERR_UNSUPPORTED otherwise).  Asynchronous on `stream`; tokens == 0 or
+ * d_out == 0 launches nothing.  y must not overlap the inputs. */
+DORA_API int dora_fused_linear_fwd(const void* x, const void* W, const void* A, const void* B, const void* bias,
+                                   const float* m, const float* n, float s, int64_t tokens, int64_t d_in,
+                                   int64_t d_out, int64_t r, dora_dtype dt, void* y, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
 /* Human-readable name of a dora_status value (static storage). */
 DORA_API const char* dora_status_string(int status);
 

@@ -200,3 +200,36 @@ def test_stream_k_partition(U, G):
                     assert idx not in seen
                     seen.add(idx)
         assert max(seen, default=0) < G + (U + kb_total - 1) // kb_total
+
+
+def test_fused_linear_argument_errors(lib):
+    f = lib.dora_fused_linear_fwd
+    ws = lib.dora_fused_linear_fwd_workspace_size(4, 16)
+    assert ws == 256
+    assert lib.dora_fused_linear_fwd_workspace_size(8192, 384) == 8192 * 384 * 2
+    # x, W, A, B, bias, m, n, s, tokens, d_in, d_out, r, dt, y, workspace, bytes, stream
+    args = [FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 0.5, 4, 64, 64, 16, D.DORA_BF16, FAKE, FAKE, ws, None]
+
+    def call(**kw):
+        a = list(args)
+        names = ["x", "W", "A", "B", "bias", "m", "n", "s", "tokens", "d_in", "d_out", "r", "dt", "y", "ws", "wsb"]
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return f(*a)
+
+    assert call(dt=D.DORA_F32) == D.DORA_ERR_UNSUPPORTED
+    assert call(tokens=-1) == D.DORA_ERR_INVALID_ARG
+    assert call(tokens=0) == D.DORA_OK
+    assert call(d_out=0) == D.DORA_OK
+    assert call(d_in=0) == D.DORA_ERR_UNSUPPORTED
+    assert call(x=None) == D.DORA_ERR_INVALID_ARG
+    assert call(A=None) == D.DORA_ERR_INVALID_ARG
+    assert call(m=None) == D.DORA_ERR_INVALID_ARG
+    assert call(d_in=60) == D.DORA_ERR_UNSUPPORTED
+    assert call(r=12) == D.DORA_ERR_UNSUPPORTED
+    assert call(d_out=20) == D.DORA_ERR_UNSUPPORTED
+    assert call(W=MISALIGNED) == D.DORA_ERR_UNSUPPORTED
+    assert call(bias=ctypes.c_void_p(0x10001)) == D.DORA_ERR_UNSUPPORTED
+    assert call(wsb=ws - 1) == D.DORA_ERR_WORKSPACE
+    assert call(ws=None) == D.DORA_ERR_WORKSPACE
+    assert call(ws=MISALIGNED) == D.DORA_ERR_UNSUPPORTED
