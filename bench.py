@@ -214,8 +214,9 @@ def run_ours(args, rank, world, local_rank):
     e2e = run_e2e(args, D, dev, wl, W, A, B, m, base, lora, dy, n, y, d_base, d_lora, d_m, ws_n, ws_b, world)
     dense = run_dense_comparator(D, dev, W, A, B, s, ws_n) if rank == 0 else None
     batched = run_batched_context(D, dev) if rank == 0 else None
+    fused = run_fused_linear_context(D, dev, wl, W, A, B, m, n) if rank == 0 else None
     return dict(t_total=t_total, t_norm=t_norm, t_fwd=t_fwd, t_bwd=t_bwd, clocks=clocks, status=status, e2e=e2e,
-                wl=wl, dense=dense, batched=batched)
+                wl=wl, dense=dense, batched=batched, fused=fused)
 
 
 def run_dense_comparator(D, dev, W, A, B, s, ws_n, reps=10):
@@ -250,6 +251,59 @@ def run_dense_comparator(D, dev, W, A, B, s, ws_n, reps=10):
     return {"what": "row norm by materialising B A (torch matmul, bf16) vs the factored norm; context only",
             "dense_time_us": t_dense, "factored_time_us": t_factored,
             "dense_transient_bytes": dense_peak, "factored_workspace_bytes": ws_n.numel()}
+
+
+def linear_flops(T, d_in, d_out, r):
+    """Algorithmic FLOPs of the fused linear forward: x W^T and P B^T (K = d_in + r
+    over T x d_out outputs) plus P = x A^T (T x r x d_in)."""
+    return 2.0 * T * d_out * (d_in + r) + 2.0 * T * r * d_in
+
+
+def run_fused_linear_context(D, dev, wl, W, A, B, m, n, reps=10):
+    """The compose fused into the producing GEMMs (dora_fused_linear_fwd) at the
+    workload's shape (tokens x d_in -> d_out, rank r, with a bias), against the
+    unfused path a framework runs: cuBLAS x W^T (+ b), cuBLAS (x A^T) B^T, then
+    dora_compose_fwd.  Inputs and outputs (x, W, y: 134 MB each at 8192^2) are
+    larger than L2.  Context beside the step, timed with CUDA events."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(4321)
+    T = wl.tokens
+    x = torch.randn(T, wl.d_in, generator=g, device=dev).to(torch.bfloat16)
+    b = (0.1 * torch.randn(wl.d_out, generator=g, device=dev)).to(torch.bfloat16)
+    mf = m.float().contiguous()
+    y = torch.empty(T, wl.d_out, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(D.dora_fused_linear_fwd_workspace_size(T, wl.r), dtype=torch.uint8, device=dev)
+    base = torch.empty_like(y)
+    lora = torch.empty_like(y)
+
+    def fused():
+        D.dora_fused_linear_fwd(x, W, A, B, mf, n, wl.s, bias=b, y=y, workspace=ws)
+
+    def unfused():
+        torch.matmul(x, W.t(), out=base)
+        base.add_(b)
+        torch.matmul(torch.matmul(x, A.t()), B.t(), out=lora)
+        D.dora_compose_fwd(base, lora, mf, n, wl.s, y=y, bias=b)
+
+    def timed(f):
+        for _ in range(3):
+            f()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            f()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps * 1e-3
+
+    t_f = timed(fused)
+    t_u = timed(unfused)
+    F = linear_flops(T, wl.d_in, wl.d_out, wl.r)
+    return {"what": f"y = b + (m/n)(x W^T + s (x A^T) B^T) for {T} tokens, {wl.d_in} -> {wl.d_out}, r = {wl.r}, bf16, "
+                    "bias: dora_fused_linear_fwd vs cuBLAS GEMMs + dora_compose_fwd; context only",
+            "fused_us": t_f * 1e6, "unfused_us": t_u * 1e6, "flops": F, "fused_tflops": F / t_f / 1e12,
+            "speedup_vs_unfused": t_u / t_f, "gpu_launches_per_call": 2, "device_status": D.dora_device_status()}
 
 
 # the seven adapted projections of one decoder block of an 8B-class model
@@ -504,6 +558,16 @@ def build_line(args, res, N, peaks, peak_src, traffic, cpu):
         line["dense_comparator"] = res["dense"]
     if res.get("batched") is not None:
         line["many_modules"] = res["batched"]
+    if res.get("fused"):
+        fl = dict(res["fused"])
+        # ten calls back to back (~8 ms): between the burst and the sustained
+        # (seconds-long, power-capped) measured GEMM figures; both are given
+        fl["frac"] = fl["fused_tflops"] / peaks["bf16_tflops"]
+        fl["peak"] = peaks["bf16_tflops"]
+        fl["frac_of_sustained"] = fl["fused_tflops"] / peaks["bf16_tflops_sustained"]
+        fl["peak_sustained"] = peaks["bf16_tflops_sustained"]
+        fl["bound"] = "tensor"
+        line["fused_linear"] = fl
     return line
 
 
