@@ -13,6 +13,7 @@ from .dora_oracle import (  # noqa: F401
     dense_adapted_weight,
     linear_forward,
     magnitude_scale,
+    norm_backward,
     row_norm,
     row_norm_rows,
 )

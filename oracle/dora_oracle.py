@@ -78,6 +78,7 @@ __all__ = [
     "compose_backward",
     "compose_backward_columns",
     "linear_forward",
+    "norm_backward",
 ]
 
 
@@ -198,3 +199,28 @@ def linear_forward(x, W, A, B, m, n, s, bias=None, cols=None) -> np.ndarray:
     g = magnitude_scale(_f64(m)[cols], _f64(n)[cols])
     b = _bias(bias, d_out)[cols]
     return b[None, :] + g[None, :] * (x @ Wp.T)
+
+
+def norm_backward(W, A, B, s, n, d_n):
+    """Gradients of the row norms ``n_i = ||W_i + s B_i A||`` w.r.t. ``A`` and ``B``.
+
+    For the training variant that keeps the norm attached (Scaling DoRA,
+    Abstract, "gradient computation"; the DoRA summary page's Method defines
+    the norm of the adapted weight ``V = W + sBA``).  ``d_n`` is the upstream
+    gradient of the loss w.r.t. ``n`` (for the DoRA compose it is
+    ``-(m / n) * d_m``).  Chain rule on the dense definition: ``dn_i/dV_i =
+    V_i / n_i``, so with ``dV = (d_n / n)[:, None] * V``
+
+        dB = s * dV @ A.T        [d_out, r]
+        dA = s * B.T @ dV        [r, d_in]
+
+    Returns ``(dA, dB)``; ``W`` gets no gradient (frozen).  ``n`` is taken as
+    given (the forward's norms), not recomputed.
+    """
+    W, A, B = _f64(W), _f64(A), _f64(B)
+    s = float(s)
+    V = dense_adapted_weight(W, A, B, s)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        c = _f64(d_n) / _f64(n)
+    dV = c[:, None] * V
+    return s * (B.T @ dV), s * (dV @ A.T)

@@ -23,6 +23,10 @@ Method):
                      the forward definition with n held constant;
 * hand-worked      - small integer cases with exact answers worked by hand,
                      stored in tests/golden/hand_cases.json;
+* norm backward    - the gradients of the row norms into A and B equal
+                     central finite differences of an independent
+                     pure-Python row norm, and fp64 torch.autograd of
+                     ||W + sBA||_row (numpy-free);
 * layer            - the adapted layer (dense W' = W + sBA applied to x,
                      rescaled per output channel, plus b) equals pure-Python
                      loops on tiny shapes and the separately pinned compose
@@ -290,6 +294,42 @@ def pin_bias_layer(compose_forward, compose_backward, seed=6):
         d_base0, d_lora0, _ = compose_backward(dy, base, lora, m, n, s)
         assert np.array_equal(d_base, d_base0) and np.array_equal(d_lora, d_lora0)
         assert np.max(np.abs(d_base - (m / n)[None, :] * dy)) < 1e-15 * (1 + np.max(np.abs(d_base)))
+
+
+# --------------------------------------------------------- norm backward
+def pin_norm_backward(norm_backward, seed=8):
+    import torch
+
+    rng = np.random.default_rng(seed)
+    for d_out, d_in, r in ((3, 4, 2), (5, 7, 3), (4, 9, 5)):
+        W, A, B = tiny_case(rng, d_out, d_in, r)
+        d_n = rng.standard_normal(d_out)
+        for s in (0.7, -1.3):
+            n = np.array(brute_row_norm(W.tolist(), A.tolist(), B.tolist(), s))
+            dA, dB = norm_backward(W, A, B, s, n, d_n)
+            assert np.shape(dA) == (r, d_in) and np.shape(dB) == (d_out, r)
+
+            def loss(A_, B_):
+                return float(np.dot(d_n, brute_row_norm(W.tolist(), A_.tolist(), B_.tolist(), s)))
+
+            h = 1e-6
+            for (i, j) in ((0, 0), (r - 1, d_in - 1), (r // 2, d_in // 2)):
+                e = np.zeros_like(A)
+                e[i, j] = h
+                fd = (loss(A + e, B) - loss(A - e, B)) / (2 * h)
+                assert abs(fd - dA[i, j]) < 1e-6 * (1 + abs(fd)), ("dA", i, j)
+            for (i, j) in ((0, 0), (d_out - 1, r - 1), (d_out // 2, r // 2)):
+                e = np.zeros_like(B)
+                e[i, j] = h
+                fd = (loss(A, B + e) - loss(A, B - e)) / (2 * h)
+                assert abs(fd - dB[i, j]) < 1e-6 * (1 + abs(fd)), ("dB", i, j)
+
+            At = torch.tensor(A, requires_grad=True)
+            Bt = torch.tensor(B, requires_grad=True)
+            nt = torch.linalg.vector_norm(torch.tensor(W) + s * (Bt @ At), dim=1)
+            (nt * torch.tensor(d_n)).sum().backward()
+            assert np.max(np.abs(dA - At.grad.numpy())) < 1e-12 * (1 + np.max(np.abs(dA)))
+            assert np.max(np.abs(dB - Bt.grad.numpy())) < 1e-12 * (1 + np.max(np.abs(dB)))
 
 
 # ----------------------------------------------------------------- layer

@@ -31,6 +31,36 @@ def test_finite_differences():
     pins.pin_finite_differences(oracle.compose_forward, oracle.compose_backward)
 
 
+def test_norm_backward():
+    pins.pin_norm_backward(oracle.norm_backward)
+
+
+def _nb_no_s(W, A, B, s, n, d_n):
+    return oracle.norm_backward(W, A, B, 1.0, n, d_n)
+
+
+def _nb_dB_sign(W, A, B, s, n, d_n):
+    dA, dB = oracle.norm_backward(W, A, B, s, n, d_n)
+    return dA, -dB
+
+
+def _nb_no_div(W, A, B, s, n, d_n):
+    return oracle.norm_backward(W, A, B, s, np.ones(len(n)), d_n)
+
+
+def _nb_s_once(W, A, B, s, n, d_n):
+    # forgets that V itself carries s B A (uses W only inside dV)
+    W64, A64, B64 = (np.asarray(v, float) for v in (W, A, B))
+    dV = (np.asarray(d_n, float) / np.asarray(n, float))[:, None] * W64
+    return s * (B64.T @ dV), s * (dV @ A64.T)
+
+
+@pytest.mark.parametrize("mutant", [_nb_no_s, _nb_dB_sign, _nb_no_div, _nb_s_once], ids=lambda f: f.__name__)
+def test_norm_backward_mutant_is_caught(mutant):
+    with pytest.raises((AssertionError, ValueError)):
+        pins.pin_norm_backward(mutant)
+
+
 def test_layer():
     pins.pin_layer(oracle.linear_forward, oracle.compose_forward)
 
