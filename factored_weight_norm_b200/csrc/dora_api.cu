@@ -17,6 +17,7 @@
 #include "../../include/dora.h"
 #include "compose.cuh"
 #include "linear_tc.cuh"
+#include "norm_bwd.cuh"
 #include "norm_simt.cuh"
 #include "norm_tc.cuh"
 #include "norm_batched.cuh"
@@ -38,6 +39,13 @@ int linear_pair_stages(int smem_optin) {
 }
 size_t linear_pair_smem(int smem_optin) {
   return static_cast<size_t>(linear_pair_stages(smem_optin)) * kPairStageBytes + 1024 + kLinBarrierBytes;
+}
+template <typename K>
+int pair_attrs(K kernel, int smem_optin) {
+  return (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_optin) != cudaSuccess ||
+          cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess)
+             ? DORA_ERR_CUDA
+             : DORA_OK;
 }
 constexpr int kMaxGrid = 1024;                         // bound on the persistent grid
 constexpr int kMaxGramSplits = 32;
@@ -86,9 +94,9 @@ int device_info(DeviceInfo** out) {
         cudaFuncSetAttribute(gram_batched_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin) !=
             cudaSuccess)
       return DORA_ERR_CUDA;
-    if (cudaFuncSetAttribute(linear_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(linear_pair_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess)
+    if (pair_attrs(linear_pair_kernel<false, false>, d.smem_optin) ||
+        pair_attrs(linear_pair_kernel<false, true>, d.smem_optin) ||
+        pair_attrs(linear_pair_kernel<true, true>, d.smem_optin))
       return DORA_ERR_CUDA;
     {
       cudaLaunchConfig_t occ{};
@@ -102,7 +110,7 @@ int device_info(DeviceInfo** out) {
       occ.dynamicSmemBytes = linear_pair_smem(d.smem_optin);
       occ.attrs = cl;
       occ.numAttrs = 1;
-      if (cudaOccupancyMaxActiveClusters(&d.pair_clusters, linear_pair_kernel, &occ) != cudaSuccess ||
+      if (cudaOccupancyMaxActiveClusters(&d.pair_clusters, linear_pair_kernel<false, false>, &occ) != cudaSuccess ||
           d.pair_clusters < 1)
         return DORA_ERR_CUDA;
     }
@@ -241,7 +249,7 @@ int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_
   ga.partial = Gp;
   ga.status = dev->status;
   const size_t gram_smem = kGramStages * kGramStageBytes + (2 * kGramStages + 1) * 8 + 16 + 1024;
-  gram_tc_kernel<<<p.gram_tiles * ga.splits, kNormThreads, gram_smem, st>>>(tmA, ga);
+  gram_tc_kernel<<<p.gram_tiles * ga.splits, kNormThreads, gram_smem, st>>>(tmA, tmA, ga);
   if (launch_error()) return DORA_ERR_CUDA;
 
   cudaLaunchAttribute pdl[1];
@@ -742,7 +750,8 @@ int dora_fused_linear_fwd(const void* x, const void* W, const void* A, const voi
     pa.status = dev->status;
     cfg.numAttrs = 1;  // cluster shape only: ordered after everything before it on the stream
     cfg.gridDim = dim3(pairs_for(static_cast<long long>(pa.tiles_m) * pa.tiles_n));
-    if (cudaLaunchKernelEx(&cfg, linear_pair_kernel, tmX, tmA, tmX, tmA, pa) != cudaSuccess) return DORA_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, linear_pair_kernel<false, false>, tmX, tmA, tmX, tmA, pa) != cudaSuccess)
+      return DORA_ERR_CUDA;
   }
 
   // 2) y = bf16(g * [x | P] [W | B]^T + b), dependent on 1) only for the extension blocks
@@ -768,7 +777,181 @@ int dora_fused_linear_fwd(const void* x, const void* W, const void* A, const voi
   cfg.gridDim = dim3(pairs_for(static_cast<long long>(la.tiles_m) * la.tiles_n));
   const CUtensorMap& tmA2 = r > 0 ? tmP : tmX;
   const CUtensorMap& tmB2 = r > 0 ? tmB : tmW;
-  if (cudaLaunchKernelEx(&cfg, linear_pair_kernel, tmX, tmW, tmA2, tmB2, la) != cudaSuccess) return DORA_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, linear_pair_kernel<false, false>, tmX, tmW, tmA2, tmB2, la) != cudaSuccess)
+    return DORA_ERR_CUDA;
+  return launch_error();
+}
+
+
+// ---------------------------------------------------- attached-norm backward
+namespace {
+struct BwdLayout {
+  int nt, splits_max;
+  size_t off_part, off_sg, off_h, off_bt, off_bct, total;
+};
+BwdLayout bwd_layout(int64_t d_out, int64_t r) {
+  BwdLayout L{};
+  L.nt = static_cast<int>(cdiv(r, kBoxRows));
+  L.splits_max = std::max(1, std::min(kMaxGramSplits, 160 / (L.nt * L.nt)));
+  size_t off = 0;
+  L.off_part = off;
+  off = align_up(off + static_cast<size_t>(L.splits_max) * L.nt * L.nt * kBoxRows * kBoxRows * 4, 256);
+  L.off_sg = off;
+  off = align_up(off + static_cast<size_t>(r) * r * 2, 256);
+  L.off_h = off;
+  off = align_up(off + static_cast<size_t>(r) * r * 2, 256);
+  L.off_bt = off;
+  off = align_up(off + static_cast<size_t>(r) * d_out * 2, 256);
+  L.off_bct = off;
+  off = align_up(off + static_cast<size_t>(r) * d_out * 2, 256);
+  L.total = std::max<size_t>(off, 256);
+  return L;
+}
+}  // namespace
+
+size_t dora_factored_norm_bwd_workspace_size(int64_t d_out, int64_t d_in, int64_t r) {
+  if (d_out < 0 || d_in < 0 || r < 0) return 0;
+  return bwd_layout(d_out, r).total;
+}
+
+int dora_factored_norm_bwd(const void* W, const void* A, const void* B, float s, const float* n, const float* d_n,
+                           int64_t d_out, int64_t d_in, int64_t r, dora_dtype dt, float* dA, float* dB,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  if (dt != DORA_BF16) return DORA_ERR_UNSUPPORTED;
+  if (d_out < 0 || d_in < 0 || r < 0) return DORA_ERR_INVALID_ARG;
+  if (d_out > INT32_MAX / 2 || d_in > INT32_MAX / 2 || r > INT32_MAX / 2) return DORA_ERR_UNSUPPORTED;
+  if (r == 0) return DORA_OK;  // dA and dB are empty
+  if ((d_in > 0 && !dA) || (d_out > 0 && !dB)) return DORA_ERR_INVALID_ARG;
+  if (!aligned(dA, 16) || !aligned(dB, 16)) return DORA_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d_out == 0 || d_in == 0) {
+    // no rows: dA = 0; no columns: V = 0 + s B A with A empty, so dB = 0
+    float* z = d_out == 0 ? dA : dB;
+    const size_t bytes = static_cast<size_t>(r) * (d_out == 0 ? d_in : d_out) * 4;
+    if (bytes == 0) return DORA_OK;
+    return cudaMemsetAsync(z, 0, bytes, st) == cudaSuccess ? DORA_OK : DORA_ERR_CUDA;
+  }
+  if (!W || !A || !B || !n || !d_n) return DORA_ERR_INVALID_ARG;
+  if (d_in % 8 != 0 || d_out % 8 != 0 || r % 8 != 0) return DORA_ERR_UNSUPPORTED;
+  if (!aligned(W, 16) || !aligned(A, 16) || !aligned(B, 16) || !aligned(n, 4) || !aligned(d_n, 4))
+    return DORA_ERR_UNSUPPORTED;
+  const BwdLayout L = bwd_layout(d_out, r);
+  if (!workspace || workspace_bytes < L.total) return DORA_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return DORA_ERR_UNSUPPORTED;
+  DeviceInfo* dev = nullptr;
+  if (device_info(&dev)) return DORA_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* part = reinterpret_cast<float*>(ws + L.off_part);
+  __nv_bfloat16* sG = reinterpret_cast<__nv_bfloat16*>(ws + L.off_sg);
+  __nv_bfloat16* s2H = reinterpret_cast<__nv_bfloat16*>(ws + L.off_h);
+  __nv_bfloat16* Bt = reinterpret_cast<__nv_bfloat16*>(ws + L.off_bt);
+  __nv_bfloat16* Bct = reinterpret_cast<__nv_bfloat16*>(ws + L.off_bct);
+
+  CUtensorMap tmW, tmA, tmB, tmSG, tmBt, tmBct, tmH, tmWmn, tmAmn;
+  if (make_map(&tmW, W, d_out, d_in) || make_map(&tmA, A, r, d_in) || make_map(&tmB, B, d_out, r) ||
+      make_map(&tmSG, sG, r, r) || make_map(&tmBt, Bt, r, d_out) || make_map(&tmBct, Bct, r, d_out) ||
+      make_map(&tmH, s2H, r, r) || make_map(&tmWmn, W, d_out, d_in, 64) || make_map(&tmAmn, A, r, d_in, 64))
+    return DORA_ERR_CUDA;
+
+  // 1) B^T and (s c B)^T
+  norm_bwd_prep_kernel<<<dim3(static_cast<unsigned>(cdiv(d_out, 32)), static_cast<unsigned>(cdiv(r, 32))), 256, 0,
+                         st>>>(static_cast<const __nv_bfloat16*>(B), d_n, n, s, static_cast<int>(d_out),
+                               static_cast<int>(r), Bt, Bct);
+  if (launch_error()) return DORA_ERR_CUDA;
+
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  const size_t gram_smem = kGramStages * kGramStageBytes + (2 * kGramStages + 1) * 8 + 16 + 1024;
+  // split-K Gram-type product M-side x N-side^T (r x r) over kb K blocks, then
+  // the fixed-order reduction scaled by `scale` into bf16 `out`
+  auto gram_pair = [&](const CUtensorMap& mside, const CUtensorMap& nside, int kb, float scale,
+                       __nv_bfloat16* out) -> int {
+    GramArgs ga{};
+    ga.r = static_cast<int>(r);
+    ga.kb_main = kb;
+    ga.n_tiles = L.nt;
+    ga.splits = std::max(1, std::min({L.splits_max, dev->num_sms / (L.nt * L.nt), kb}));
+    ga.wait_limit = kWaitLimitCycles;
+    ga.partial = part;
+    ga.status = dev->status;
+    gram_tc_kernel<<<L.nt * L.nt * ga.splits, kNormThreads, gram_smem, st>>>(mside, nside, ga);
+    if (launch_error()) return DORA_ERR_CUDA;
+    cudaLaunchConfig_t cfg{};
+    cfg.stream = st;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    const long long rr = static_cast<long long>(r) * r;
+    cfg.gridDim = dim3(static_cast<unsigned>(std::max<long long>(1, std::min<long long>(cdiv(rr, 1024), 4 * dev->num_sms))));
+    cfg.blockDim = dim3(256);
+    if (cudaLaunchKernelEx(&cfg, gram_reduce_kernel, static_cast<const float*>(part), ga.splits, static_cast<int>(r),
+                           scale, out, static_cast<int*>(nullptr), 0) != cudaSuccess)
+      return DORA_ERR_CUDA;
+    return DORA_OK;
+  };
+
+  cudaLaunchAttribute attrs[2];
+  attrs[0].id = cudaLaunchAttributeClusterDimension;
+  attrs[0].val.clusterDim.x = 2;
+  attrs[0].val.clusterDim.y = 1;
+  attrs[0].val.clusterDim.z = 1;
+  attrs[1] = pdl[0];
+  cudaLaunchConfig_t pcfg{};
+  pcfg.stream = st;
+  pcfg.attrs = attrs;
+  pcfg.numAttrs = 2;
+  pcfg.blockDim = dim3(kLinThreads);
+  pcfg.dynamicSmemBytes = linear_pair_smem(dev->smem_optin);
+  const int stages = linear_pair_stages(dev->smem_optin);
+  if (stages < 2) return DORA_ERR_UNSUPPORTED;
+  auto pair_grid = [&](const LinearArgs& la) {
+    return dim3(static_cast<unsigned>(2 * std::min<long long>(dev->pair_clusters,
+                                                              static_cast<long long>(la.tiles_m) * la.tiles_n)));
+  };
+
+  // 2) s G, then dB = s c * ([W | B] [A | s G]^T)
+  if (int e = gram_pair(tmA, tmA, static_cast<int>(cdiv(d_in, kBK)), s, sG)) return e;
+  LinearArgs lb{};
+  lb.M = static_cast<int>(d_out);
+  lb.N = static_cast<int>(r);
+  lb.kb_main = static_cast<int>(cdiv(d_in, kLinBK));
+  lb.kb_total = lb.kb_main + static_cast<int>(cdiv(r, kLinBK));
+  lb.tiles_m = static_cast<int>(cdiv(d_out, kPairBM));
+  lb.tiles_n = static_cast<int>(cdiv(r, kPairBN));
+  lb.stages = stages;
+  lb.stage_bytes = kPairStageBytes;
+  lb.alpha = s;
+  lb.rs_num = d_n;
+  lb.rs_den = n;
+  lb.out = dB;
+  lb.ldo = r;
+  lb.ext_waits = 1;
+  lb.wait_limit = kWaitLimitCycles;
+  lb.status = dev->status;
+  pcfg.gridDim = pair_grid(lb);
+  if (cudaLaunchKernelEx(&pcfg, linear_pair_kernel<false, true>, tmW, tmA, tmB, tmSG, lb) != cudaSuccess)
+    return DORA_ERR_CUDA;
+
+  // 3) s^2 H = s (s c B)^T B, then dA = [(s c B)^T | s^2 H] [W ; A]
+  if (int e = gram_pair(tmBct, tmBt, static_cast<int>(cdiv(d_out, kBK)), s, s2H)) return e;
+  LinearArgs la{};
+  la.M = static_cast<int>(r);
+  la.N = static_cast<int>(d_in);
+  la.kb_main = static_cast<int>(cdiv(d_out, kLinBK));
+  la.kb_total = la.kb_main + static_cast<int>(cdiv(r, kLinBK));
+  la.tiles_m = static_cast<int>(cdiv(r, kPairBM));
+  la.tiles_n = static_cast<int>(cdiv(d_in, kPairBN));
+  la.stages = stages;
+  la.stage_bytes = kPairStageBytes;
+  la.alpha = 1.f;
+  la.out = dA;
+  la.ldo = d_in;
+  la.ext_waits = 1;
+  la.wait_limit = kWaitLimitCycles;
+  la.status = dev->status;
+  pcfg.gridDim = pair_grid(la);
+  if (cudaLaunchKernelEx(&pcfg, linear_pair_kernel<true, true>, tmBct, tmWmn, tmH, tmAmn, la) != cudaSuccess)
+    return DORA_ERR_CUDA;
   return launch_error();
 }
 

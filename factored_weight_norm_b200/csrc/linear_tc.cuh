@@ -57,8 +57,10 @@ struct LinearArgs {
   float alpha;             // uniform scale of the product
   const float* m;          // per-column g = m / n, or null (g = 1)
   const float* n;
+  const float* rs_num;     // per-row scale rs_num / rs_den, or null (1)
+  const float* rs_den;
   const __nv_bfloat16* bias;  // per-column bias, or null
-  __nv_bfloat16* out;      // [M, ldo] row-major
+  void* out;               // [M, ldo] row-major, bf16 or fp32 (kernel template)
   long long ldo;
   int ext_waits;           // 1: the extension operands come from the preceding grid
   long long wait_limit;
@@ -99,6 +101,10 @@ constexpr int kPairKps = 2;  // 64-deep K blocks per ring stage (one barrier rou
 // per stage: kPairKps boxes of 128 A-side rows, then kPairKps boxes of 128 B-side rows
 constexpr uint32_t kPairStageBytes = 2 * kPairKps * kLinABytes;
 
+// B_MN: the B-side operand is stored N-contiguous (its rows run along K), as
+// W is for a contraction over d_out; it is loaded as two 64-column boxes per
+// K block and read through MN-major descriptors.  OUT_F32: fp32 output.
+template <bool B_MN, bool OUT_F32>
 __global__ void __launch_bounds__(kLinThreads, 1)
     linear_pair_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
                        const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
@@ -191,13 +197,25 @@ __global__ void __launch_bounds__(kLinThreads, 1)
         }
         const uint32_t dst = base_s + stage * kPairStageBytes;
         const uint32_t bar = full_leader + static_cast<uint32_t>(stage) * 8u;
-        if (lane < 2 * kPairKps) {
-          const int i = lane % kPairKps;
+        if (lane < kPairKps) {
+          const int kb = kb0 + lane;
+          const bool ext = kb >= a.kb_main && a.kb_total > a.kb_main;
+          const int xk = (ext ? kb - a.kb_main : kb) * kLinBK;
+          tma_load_2d_pair(dst + lane * kLinABytes, ext ? &tmA2 : &tmA1, bar, xk, ya);
+        } else if (!B_MN && lane < 2 * kPairKps) {
+          const int i = lane - kPairKps;
           const int kb = kb0 + i;
           const bool ext = kb >= a.kb_main && a.kb_total > a.kb_main;
           const int xk = (ext ? kb - a.kb_main : kb) * kLinBK;
-          if (lane < kPairKps) tma_load_2d_pair(dst + i * kLinABytes, ext ? &tmA2 : &tmA1, bar, xk, ya);
-          else tma_load_2d_pair(dst + (kPairKps + i) * kLinABytes, ext ? &tmB2 : &tmB1, bar, xk, yb);
+          tma_load_2d_pair(dst + (kPairKps + i) * kLinABytes, ext ? &tmB2 : &tmB1, bar, xk, yb);
+        } else if (B_MN && lane < 3 * kPairKps) {
+          // K block i: columns yb.. and yb + 64.. of rows (K) kb * 64 .., two 8 KB boxes
+          const int i = (lane - kPairKps) >> 1, h = (lane - kPairKps) & 1;
+          const int kb = kb0 + i;
+          const bool ext = kb >= a.kb_main && a.kb_total > a.kb_main;
+          const int yk = (ext ? kb - a.kb_main : kb) * kLinBK;
+          tma_load_2d_pair(dst + (kPairKps + i) * kLinABytes + h * (kLinABytes / 2), ext ? &tmB2 : &tmB1, bar,
+                           yb + 64 * h, yk);
         }
         parity_bits = (parity_bits & ~(1u << stage)) | (phase << stage);
         filled_mask |= 1u << stage;
@@ -218,9 +236,12 @@ __global__ void __launch_bounds__(kLinThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      const uint32_t idesc = idesc_bf16_f32(kPairBM, kPairBN);
+      const uint32_t idesc = idesc_bf16_f32(kPairBM, kPairBN) | (B_MN ? kIdescBMnMajor : 0u);
       const uint64_t desc0 = sw128_kmajor_desc(base_s);
       const uint64_t desc_step = kPairStageBytes >> 4;
+      // MN-major B: the two 64-column boxes of a K block are 8 KB apart (the
+      // leading byte offset); 8-row K groups are 1024 B apart; 16 K rows per MMA
+      const uint64_t bdesc_mn0 = sw128_mn_desc(base_s + kPairKps * kLinABytes, kLinABytes / 2);
       int it = 0;
       for (int t = cid; t < n_tiles && ok; t += n_pairs, ++it) {
         const int ab = it & 1;
@@ -238,13 +259,16 @@ __global__ void __launch_bounds__(kLinThreads, 1)
           }
           tc_fence_after();
           const uint64_t adesc = desc0 + static_cast<uint64_t>(stage) * desc_step;
-          const uint64_t bdesc = adesc + ((kPairKps * kLinABytes) >> 4);
+          const uint64_t bdesc = B_MN ? bdesc_mn0 + static_cast<uint64_t>(stage) * desc_step
+                                      : adesc + ((kPairKps * kLinABytes) >> 4);
+          // K-major: +32 B along K inside the swizzled row; MN-major: +16 rows of 128 B
+          constexpr uint64_t kb_step = B_MN ? (16 * 128) >> 4 : 2;
 #pragma unroll
           for (int i = 0; i < kPairKps; ++i)
 #pragma unroll
             for (int k = 0; k < kLinBK / 16; ++k)
-              mma_bf16_pair(d, adesc + i * (kLinABytes >> 4) + 2 * k, bdesc + i * (kLinABytes >> 4) + 2 * k, idesc,
-                            (kb0 > 0 || i > 0 || k > 0) ? 1u : 0u);
+              mma_bf16_pair(d, adesc + i * (kLinABytes >> 4) + 2 * k, bdesc + i * (kLinABytes >> 4) + kb_step * k,
+                            idesc, (kb0 > 0 || i > 0 || k > 0) ? 1u : 0u);
           mma_commit_pair(&empty[stage], 0x3);
           if (++stage == a.stages) {
             stage = 0;
@@ -272,7 +296,7 @@ __global__ void __launch_bounds__(kLinThreads, 1)
       tc_fence_after();
       const long long row = static_cast<long long>(tm) * kPairBM + rank * kLinBM + q * 32 + lane;
       const bool row_ok = row < a.M;
-      __nv_bfloat16* dst_row = a.out + row * a.ldo;
+      const float rscale = (row_ok && a.rs_num) ? __ldg(a.rs_num + row) / __ldg(a.rs_den + row) : 1.f;
 #pragma unroll 1
       for (int c = 0; c < kPairBN / 32; ++c) {
         const int col0 = tn * kPairBN + c * 32;
@@ -287,17 +311,27 @@ __global__ void __launch_bounds__(kLinThreads, 1)
         }
 #pragma unroll
         for (int e = 0; e < 32; ++e)
-          v[e] = fmaf(v[e], __shfl_sync(0xffffffffu, gl, e), __shfl_sync(0xffffffffu, bl, e));
+          v[e] = fmaf(v[e] * rscale, __shfl_sync(0xffffffffu, gl, e), __shfl_sync(0xffffffffu, bl, e));
         if (row_ok) {
+          if (OUT_F32) {
+            float* dst_row = static_cast<float*>(a.out) + row * a.ldo;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            if (col0 + 8 * j < a.N) {
-              uint4 pk;
-              pk.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
-              pk.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
-              pk.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
-              pk.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
-              *reinterpret_cast<uint4*>(dst_row + col0 + 8 * j) = pk;
+            for (int j = 0; j < 8; ++j)
+              if (col0 + 4 * j < a.N)
+                *reinterpret_cast<float4*>(dst_row + col0 + 4 * j) =
+                    make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+          } else {
+            __nv_bfloat16* dst_row = static_cast<__nv_bfloat16*>(a.out) + row * a.ldo;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              if (col0 + 8 * j < a.N) {
+                uint4 pk;
+                pk.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
+                pk.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+                pk.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+                pk.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+                *reinterpret_cast<uint4*>(dst_row + col0 + 8 * j) = pk;
+              }
             }
           }
         }

@@ -510,7 +510,7 @@ constexpr int kGramStages = 3;
 constexpr uint32_t kGramStageBytes = 2 * kGramKPerStage * kBoxBytes;
 
 __global__ void __launch_bounds__(kNormThreads, 1)
-    gram_tc_kernel(const __grid_constant__ CUtensorMap tmA, const GramArgs a) {
+    gram_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const GramArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   const uint32_t base_s = (raw_s + 1023u) & ~1023u;
@@ -544,7 +544,10 @@ __global__ void __launch_bounds__(kNormThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) tma_prefetch_desc(&tmA);
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 128);
     tmem_relinquish();
@@ -571,8 +574,8 @@ __global__ void __launch_bounds__(kNormThreads, 1)
       if (!__shfl_sync(0xffffffffu, got, 0)) break;
       __syncwarp();
       if (lane < 2 * nk)
-        tma_load_2d(base_s + stage * kGramStageBytes + lane * kBoxBytes, &tmA, &full[stage], (kb0 + (lane >> 1)) * kBK,
-                    ((lane & 1) ? ni : mi) * kBoxRows);
+        tma_load_2d(base_s + stage * kGramStageBytes + lane * kBoxBytes, (lane & 1) ? &tmB : &tmA, &full[stage],
+                    (kb0 + (lane >> 1)) * kBK, ((lane & 1) ? ni : mi) * kBoxRows);
       parity_bits = (parity_bits & ~(1u << stage)) | (phase << stage);
       filled_mask |= 1u << stage;
       if (++stage == kGramStages) {

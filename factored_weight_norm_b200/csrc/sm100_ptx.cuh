@@ -213,6 +213,23 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
   return d;
 }
 
+// Shared-memory matrix descriptor for an MN-major operand tile stored with the
+// 128-byte swizzle: each K row is 128 bytes (64 bf16 along M or N), 8-row K
+// groups are 1024 bytes apart (stride byte offset), and successive 64-wide
+// M/N blocks are `lbo_bytes` apart (leading byte offset).
+__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t smem_addr, uint32_t lbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+
+// Instruction-descriptor bit marking the B operand MN-major (transposed).
+constexpr uint32_t kIdescBMnMajor = 1u << 16;
+
 // Instruction descriptor: kind::f16 with bf16 A/B, fp32 D, both K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4)                                 // D format: fp32

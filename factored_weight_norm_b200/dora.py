@@ -67,6 +67,12 @@ SIGNATURES = {
     "dora_selftest_timeout": (ctypes.c_int, [_i64, _c_void_p]),
     "dora_factored_norm_batched_workspace_size": (_size, [_problems_p, ctypes.c_int, ctypes.c_int]),
     "dora_factored_norm_batched": (ctypes.c_int, [_problems_p, ctypes.c_int, ctypes.c_int, _c_void_p, _size, _c_void_p]),
+    "dora_factored_norm_bwd_workspace_size": (_size, [_i64, _i64, _i64]),
+    "dora_factored_norm_bwd": (
+        ctypes.c_int,
+        [_c_void_p, _c_void_p, _c_void_p, _f32, _c_void_p, _c_void_p, _i64, _i64, _i64, ctypes.c_int, _c_void_p,
+         _c_void_p, _c_void_p, _size, _c_void_p],
+    ),
     "dora_fused_linear_fwd_workspace_size": (_size, [_i64, _i64]),
     "dora_fused_linear_fwd": (
         ctypes.c_int,
@@ -339,3 +345,34 @@ def dora_fused_linear_fwd(x, W, A, B, m, n, s: float, bias=None, y=None, workspa
     )
     _check(st, "dora_fused_linear_fwd")
     return y
+
+
+def dora_factored_norm_bwd_workspace_size(d_out: int, d_in: int, r: int) -> int:
+    return int(lib().dora_factored_norm_bwd_workspace_size(d_out, d_in, r))
+
+
+def dora_factored_norm_bwd(W, A, B, s: float, n, d_n, dA=None, dB=None, workspace=None, stream=None):
+    """(dA, dB): gradients of n_i = ||W_i + s B_i A|| into A and B (fp32), given d_n = dL/dn."""
+    _dense_cuda(W, A, B, n, d_n, dA, dB, workspace)
+    d_out, d_in = W.shape
+    r = A.shape[0]
+    if A.shape != (r, d_in) or B.shape != (d_out, r) or n.shape != (d_out,) or d_n.shape != (d_out,):
+        raise ValueError("shape mismatch in dora_factored_norm_bwd")
+    for t in (W, A, B):
+        if t.dtype != torch.bfloat16:
+            raise TypeError("W, A and B must be bf16")
+    if n.dtype != torch.float32 or d_n.dtype != torch.float32:
+        raise TypeError("n and d_n must be fp32")
+    if dA is None:
+        dA = torch.empty(r, d_in, dtype=torch.float32, device=W.device)
+    if dB is None:
+        dB = torch.empty(d_out, r, dtype=torch.float32, device=W.device)
+    need = dora_factored_norm_bwd_workspace_size(d_out, d_in, r)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
+    st = lib().dora_factored_norm_bwd(
+        _ptr(W), _ptr(A), _ptr(B), float(s), _ptr(n), _ptr(d_n), d_out, d_in, r, DORA_BF16, _ptr(dA), _ptr(dB),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream),
+    )
+    _check(st, "dora_factored_norm_bwd")
+    return dA, dB

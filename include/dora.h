@@ -182,6 +182,38 @@ DORA_API int dora_compose_bwd_noalloc(const void* dy, const void* base_out, cons
                                       const float* m, const float* n, float s, int64_t tokens, int64_t d_out,
                                       dora_dtype dt, void* d_base, void* d_lora, float* d_m, void* stream);
 
+/* Bytes of workspace dora_factored_norm_bwd needs: O(r^2 + r d_out), no
+ * d_out x d_in term (the Gram partial tiles, s G and s^2 H in bf16, and two
+ * [r, d_out] bf16 copies of B). */
+DORA_API size_t dora_factored_norm_bwd_workspace_size(int64_t d_out, int64_t d_in, int64_t r);
+
+/* Gradients of the row norms n_i = ||W_i + s B_i A|| into A and B, for
+ * training with the norm kept attached (Scaling DoRA, Abstract: the factored
+ * norm's "gradient computation"; the default DoRA backward, dora_compose_bwd,
+ * holds n constant).  With c = d_n / n and never forming B A:
+ *
+ *   dB = s c * (W A^T + s B G),            G = A A^T
+ *   dA = s (c * B)^T W + s^2 H A,          H = (c * B)^T B
+ *
+ * computed as a Gram product and a CTA-pair tcgen05 GEMM for each (dB:
+ * [W | B] [A | s G]^T with a per-row epilogue scale; dA: [(s c B)^T | s^2 H]
+ * [W ; A], W read N-contiguous), G, H and (s c B)^T rounded to bf16, fp32
+ * accumulation.
+ *
+ * W: [d_out, d_in]; A: [r, d_in]; B: [d_out, r]; bf16, row-major, 16-byte
+ * aligned; d_in, d_out, r multiples of 8.  n: fp32 [d_out], the forward's
+ * norms (not recomputed); d_n: fp32 [d_out], the upstream gradient of n (for
+ * the DoRA compose y = (m / n) (base + s lora) it is -(m / n) * d_m).  dA:
+ * fp32 [r, d_in]; dB: fp32 [d_out, r]; both overwritten with the gradients
+ * through the norm alone (the caller adds the LoRA path's own gradients); W
+ * gets none.  r = 0 does nothing; d_out = 0 zeroes dA; d_in = 0 zeroes dB.
+ * workspace: at least dora_factored_norm_bwd_workspace_size() bytes,
+ * 256-byte aligned, contents ignored.  Only DORA_BF16.  Asynchronous on
+ * `stream` (six launches). */
+DORA_API int dora_factored_norm_bwd(const void* W, const void* A, const void* B, float s, const float* n,
+                                    const float* d_n, int64_t d_out, int64_t d_in, int64_t r, dora_dtype dt,
+                                    float* dA, float* dB, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Bytes of workspace dora_fused_linear_fwd needs: the [tokens, r] bf16
  * intermediate P = s * x A^T (at least 256). */
 DORA_API size_t dora_fused_linear_fwd_workspace_size(int64_t tokens, int64_t r);

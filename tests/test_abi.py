@@ -233,3 +233,37 @@ def test_fused_linear_argument_errors(lib):
     assert call(wsb=ws - 1) == D.DORA_ERR_WORKSPACE
     assert call(ws=None) == D.DORA_ERR_WORKSPACE
     assert call(ws=MISALIGNED) == D.DORA_ERR_UNSUPPORTED
+
+
+def test_norm_bwd_argument_errors(lib):
+    f = lib.dora_factored_norm_bwd
+    ws = lib.dora_factored_norm_bwd_workspace_size(64, 128, 16)
+    # W, A, B, s, n, d_n, d_out, d_in, r, dt, dA, dB, workspace, bytes, stream
+    args = [FAKE, FAKE, FAKE, 0.5, FAKE, FAKE, 64, 128, 16, D.DORA_BF16, FAKE, FAKE, FAKE, ws, None]
+    names = ["W", "A", "B", "s", "n", "d_n", "d_out", "d_in", "r", "dt", "dA", "dB", "ws", "wsb"]
+
+    def call(**kw):
+        a = list(args)
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return f(*a)
+
+    assert call(dt=D.DORA_F32) == D.DORA_ERR_UNSUPPORTED
+    assert call(r=-1) == D.DORA_ERR_INVALID_ARG
+    assert call(r=0) == D.DORA_OK            # empty gradients, nothing launched
+    assert call(dA=None) == D.DORA_ERR_INVALID_ARG
+    assert call(W=None) == D.DORA_ERR_INVALID_ARG
+    assert call(d_n=None) == D.DORA_ERR_INVALID_ARG
+    assert call(d_out=60) == D.DORA_ERR_UNSUPPORTED
+    assert call(r=12) == D.DORA_ERR_UNSUPPORTED
+    assert call(A=MISALIGNED) == D.DORA_ERR_UNSUPPORTED
+    assert call(dB=MISALIGNED) == D.DORA_ERR_UNSUPPORTED
+    assert call(wsb=ws - 1) == D.DORA_ERR_WORKSPACE
+    assert call(ws=None) == D.DORA_ERR_WORKSPACE
+
+
+def test_norm_bwd_workspace_has_no_dense_term(lib):
+    for d_out, d_in, r in ((8192, 8192, 384), (27648, 5120, 384), (4096, 4096, 64)):
+        ws = lib.dora_factored_norm_bwd_workspace_size(d_out, d_in, r)
+        assert ws < d_out * d_in * 2 // 4  # O(r d_out + r^2): 22.6 MB vs the dense 134 MB at 8192^2, r = 384
+        assert lib.dora_factored_norm_bwd_workspace_size(d_out, 2 * d_in, r) == ws  # independent of d_in

@@ -1,0 +1,110 @@
+"""dora_factored_norm_bwd (gradients of the row norms into A and B) vs the oracle.
+
+The oracle differentiates ||W + sBA||_row on the dense definition in fp64.
+The GPU rounds (s c B)^T, s G and s^2 H to bf16 and accumulates in fp32, so
+an element may be off by a small multiple of 2^-9 of the typical magnitude
+of its contraction: the bar is 1e-2 |ref| + 5e-3 max|ref| per output, written
+below.  The 8192 x 8192, r = 384 shape is checked on sampled rows of dB and
+columns of dA (dB's rows depend only on the same rows of W and B; dA's columns
+only on the same columns of W and A, so the oracle is called on those slices).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from factored_weight_norm_b200 import dora as D
+from factored_weight_norm_b200 import workloads as wlmod
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+RTOL, MTOL = 1e-2, 5e-3
+
+
+def assert_grad_close(got, ref, what):
+    got, ref = P.f64(got), np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    bound = RTOL * np.abs(ref) + MTOL * np.max(np.abs(ref))
+    bad = np.abs(got - ref) > bound
+    if bad.any():
+        idx = tuple(np.argwhere(bad)[0])
+        raise AssertionError(f"{what}: {int(bad.sum())} of {bad.size} outside 1e-2|ref| + 5e-3 max|ref|; "
+                             f"first at {idx}: gpu {got[idx]!r} ref {ref[idx]!r}")
+
+
+def _case(d_out, d_in, r, s, seed=13):
+    wl = wlmod.Workload(f"nb_{d_out}x{d_in}_r{r}", d_out, d_in, r, s, 64, "bf16", 0.02, 0.01, 1e-3, seed)
+    W, A, B, _ = wlmod.make_weights(wl, DEV)
+    n = torch.linalg.vector_norm(W.float() + s * (B.float() @ A.float()), dim=1).contiguous()
+    g = torch.Generator(device="cpu").manual_seed(seed + 1)
+    d_n = torch.randn(d_out, generator=g).to(DEV)
+    return W, A, B, n, d_n
+
+
+SMALL = [(128, 64, 16), (256, 512, 64), (296, 520, 48), (1000, 1000, 128), (512, 1024, 384), (264, 4104, 512),
+         (200, 328, 272)]
+
+
+@pytest.mark.parametrize("shape", SMALL, ids=lambda t: "x".join(map(str, t)))
+@pytest.mark.parametrize("s", [0.5, -2.0])
+def test_norm_bwd_small(shape, s):
+    d_out, d_in, r = shape
+    W, A, B, n, d_n = _case(d_out, d_in, r, s)
+    dA, dB = D.dora_factored_norm_bwd(W, A, B, s, n, d_n)
+    torch.cuda.synchronize()
+    assert D.dora_device_status() == D.DORA_OK
+    rA, rB = oracle.norm_backward(P.f64(W), P.f64(A), P.f64(B), s, P.f64(n), P.f64(d_n))
+    assert_grad_close(dA, rA, "dA")
+    assert_grad_close(dB, rB, "dB")
+
+
+def test_norm_bwd_matches_torch_autograd_of_the_dense_norm():
+    # an independent GPU check: fp32 autograd through ||W + sBA||_row
+    d_out, d_in, r, s = 512, 768, 128, 0.75
+    W, A, B, _, d_n = _case(d_out, d_in, r, s, seed=21)
+    A32 = A.float().requires_grad_()
+    B32 = B.float().requires_grad_()
+    nt = torch.linalg.vector_norm(W.float() + s * (B32 @ A32), dim=1)
+    (nt * d_n).sum().backward()
+    dA, dB = D.dora_factored_norm_bwd(W, A, B, s, nt.detach().contiguous(), d_n)
+    torch.cuda.synchronize()
+    assert_grad_close(dA, P.f64(A32.grad), "dA vs autograd")
+    assert_grad_close(dB, P.f64(B32.grad), "dB vs autograd")
+
+
+def test_norm_bwd_headline_sampled():
+    wl = wlmod.HEADLINE
+    W, A, B, _ = wlmod.make_weights(wl, DEV)
+    n = D.dora_factored_norm(W, A, B, wl.s)
+    g = torch.Generator(device=DEV).manual_seed(3)
+    d_n = torch.randn(wl.d_out, generator=g, device=DEV)
+    dA, dB = D.dora_factored_norm_bwd(W, A, B, wl.s, n, d_n)
+    torch.cuda.synchronize()
+    assert D.dora_device_status() == D.DORA_OK
+    W64, A64, B64, n64, dn64 = P.f64(W), P.f64(A), P.f64(B), P.f64(n), P.f64(d_n)
+    rows = np.array([0, 1, 127, 128, 4095, 8191])
+    _, rB = oracle.norm_backward(W64[rows], A64, B64[rows], wl.s, n64[rows], dn64[rows])
+    assert_grad_close(P.f64(dB)[rows], rB, "dB rows")
+    cols = np.array([0, 63, 64, 255, 256, 5000, 8191])
+    rA, _ = oracle.norm_backward(W64[:, cols], A64[:, cols], B64, wl.s, n64, dn64)
+    assert_grad_close(P.f64(dA)[:, cols], rA, "dA columns")
+
+
+def test_norm_bwd_degenerate_sizes_and_determinism():
+    W, A, B, n, d_n = _case(256, 512, 64, 0.5)
+    a1, b1 = D.dora_factored_norm_bwd(W, A, B, 0.5, n, d_n)
+    a2, b2 = D.dora_factored_norm_bwd(W, A, B, 0.5, n, d_n)
+    torch.cuda.synchronize()
+    assert torch.equal(a1, a2) and torch.equal(b1, b2)  # fixed summation order
+    # d_n = 0: both gradients vanish exactly
+    z = torch.zeros_like(d_n)
+    a0, b0 = D.dora_factored_norm_bwd(W, A, B, 0.5, n, z)
+    torch.cuda.synchronize()
+    assert not a0.any() and not b0.any()
+    # no output rows: dA = 0 (written, not left as it was)
+    dA = torch.full((64, 512), 7.0, device=DEV)
+    D.dora_factored_norm_bwd(W[:0], A, B[:0], 0.5, n[:0], d_n[:0], dA=dA)
+    torch.cuda.synchronize()
+    assert not dA.any()
