@@ -40,6 +40,21 @@ int linear_pair_stages(int smem_optin) {
 size_t linear_pair_smem(int smem_optin) {
   return static_cast<size_t>(linear_pair_stages(smem_optin)) * kPairStageBytes + 1024 + kLinBarrierBytes;
 }
+// Pair tile width along N for an output of N columns: the one of 256, 192,
+// 128 that pads N least (the wider on a tie), e.g. r = 384 -> 2 x 192.
+int pick_bn(long long N) {
+  int best = 256;
+  long long waste = (N + 255) / 256 * 256 - N;
+  for (int bn : {192, 128}) {
+    const long long w = (N + bn - 1) / bn * bn - N;
+    if (w < waste) {
+      waste = w;
+      best = bn;
+    }
+  }
+  return best;
+}
+
 template <typename K>
 int pair_attrs(K kernel, int smem_optin) {
   return (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_optin) != cudaSuccess ||
@@ -699,7 +714,7 @@ int dora_fused_linear_fwd(const void* x, const void* W, const void* A, const voi
   if (!aligned(x, 16) || !aligned(W, 16) || !aligned(A, 16) || !aligned(B, 16) || !aligned(y, 16) ||
       !aligned(bias, 2) || !aligned(m, 4) || !aligned(n, 4))
     return DORA_ERR_UNSUPPORTED;
-  if (cdiv(tokens, kPairBM) * cdiv(d_out, kPairBN) > INT32_MAX) return DORA_ERR_UNSUPPORTED;
+  if (cdiv(tokens, kPairBM) * cdiv(d_out, 128) > INT32_MAX) return DORA_ERR_UNSUPPORTED;
   const size_t need = dora_fused_linear_fwd_workspace_size(tokens, r);
   if (r > 0 && (!workspace || workspace_bytes < need)) return DORA_ERR_WORKSPACE;
   if (r > 0 && !aligned(workspace, 256)) return DORA_ERR_UNSUPPORTED;
@@ -708,9 +723,12 @@ int dora_fused_linear_fwd(const void* x, const void* W, const void* A, const voi
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   __nv_bfloat16* P = static_cast<__nv_bfloat16*>(workspace);
 
+  // B-side boxes hold the bn / 2 rows one CTA of a pair owns
+  const int bn_p = r > 0 ? pick_bn(r) : 256, bn_y = pick_bn(d_out);
   CUtensorMap tmX, tmW, tmA, tmP, tmB;
-  if (make_map(&tmX, x, tokens, d_in) || make_map(&tmW, W, d_out, d_in)) return DORA_ERR_CUDA;
-  if (r > 0 && (make_map(&tmA, A, r, d_in) || make_map(&tmP, P, tokens, r) || make_map(&tmB, B, d_out, r)))
+  if (make_map(&tmX, x, tokens, d_in) || make_map(&tmW, W, d_out, d_in, bn_y / 2)) return DORA_ERR_CUDA;
+  if (r > 0 && (make_map(&tmA, A, r, d_in, bn_p / 2) || make_map(&tmP, P, tokens, r) ||
+                make_map(&tmB, B, d_out, r, bn_y / 2)))
     return DORA_ERR_CUDA;
   const int kb_main = static_cast<int>(cdiv(d_in, kLinBK));
   const int stages = linear_pair_stages(dev->smem_optin);
@@ -740,7 +758,8 @@ int dora_fused_linear_fwd(const void* x, const void* W, const void* A, const voi
     pa.N = static_cast<int>(r);
     pa.kb_main = pa.kb_total = kb_main;
     pa.tiles_m = static_cast<int>(tiles_m2);
-    pa.tiles_n = static_cast<int>(cdiv(r, kPairBN));
+    pa.bn = bn_p;
+    pa.tiles_n = static_cast<int>(cdiv(r, bn_p));
     pa.stages = stages;
     pa.stage_bytes = kPairStageBytes;
     pa.alpha = s;
@@ -761,7 +780,8 @@ int dora_fused_linear_fwd(const void* x, const void* W, const void* A, const voi
   la.kb_main = kb_main;
   la.kb_total = kb_main + static_cast<int>(cdiv(r, kLinBK));
   la.tiles_m = static_cast<int>(tiles_m2);
-  la.tiles_n = static_cast<int>(cdiv(d_out, kPairBN));
+  la.bn = bn_y;
+  la.tiles_n = static_cast<int>(cdiv(d_out, bn_y));
   la.stages = stages;
   la.stage_bytes = kPairStageBytes;
   la.alpha = 1.f;
@@ -847,10 +867,12 @@ int dora_factored_norm_bwd(const void* W, const void* A, const void* B, float s,
   __nv_bfloat16* Bt = reinterpret_cast<__nv_bfloat16*>(ws + L.off_bt);
   __nv_bfloat16* Bct = reinterpret_cast<__nv_bfloat16*>(ws + L.off_bct);
 
-  CUtensorMap tmW, tmA, tmB, tmSG, tmBt, tmBct, tmH, tmWmn, tmAmn;
-  if (make_map(&tmW, W, d_out, d_in) || make_map(&tmA, A, r, d_in) || make_map(&tmB, B, d_out, r) ||
-      make_map(&tmSG, sG, r, r) || make_map(&tmBt, Bt, r, d_out) || make_map(&tmBct, Bct, r, d_out) ||
-      make_map(&tmH, s2H, r, r) || make_map(&tmWmn, W, d_out, d_in, 64) || make_map(&tmAmn, A, r, d_in, 64))
+  const int bn_b = pick_bn(r), bn_a = pick_bn(d_in);
+  CUtensorMap tmW, tmA, tmAb, tmB, tmSG, tmBt, tmBct, tmH, tmWmn, tmAmn;
+  if (make_map(&tmW, W, d_out, d_in) || make_map(&tmA, A, r, d_in) || make_map(&tmAb, A, r, d_in, bn_b / 2) ||
+      make_map(&tmB, B, d_out, r) || make_map(&tmSG, sG, r, r, bn_b / 2) || make_map(&tmBt, Bt, r, d_out) ||
+      make_map(&tmBct, Bct, r, d_out) || make_map(&tmH, s2H, r, r) || make_map(&tmWmn, W, d_out, d_in, 64) ||
+      make_map(&tmAmn, A, r, d_in, 64))
     return DORA_ERR_CUDA;
 
   // 1) B^T and (s c B)^T
@@ -917,7 +939,8 @@ int dora_factored_norm_bwd(const void* W, const void* A, const void* B, float s,
   lb.kb_main = static_cast<int>(cdiv(d_in, kLinBK));
   lb.kb_total = lb.kb_main + static_cast<int>(cdiv(r, kLinBK));
   lb.tiles_m = static_cast<int>(cdiv(d_out, kPairBM));
-  lb.tiles_n = static_cast<int>(cdiv(r, kPairBN));
+  lb.bn = bn_b;
+  lb.tiles_n = static_cast<int>(cdiv(r, bn_b));
   lb.stages = stages;
   lb.stage_bytes = kPairStageBytes;
   lb.alpha = s;
@@ -929,7 +952,7 @@ int dora_factored_norm_bwd(const void* W, const void* A, const void* B, float s,
   lb.wait_limit = kWaitLimitCycles;
   lb.status = dev->status;
   pcfg.gridDim = pair_grid(lb);
-  if (cudaLaunchKernelEx(&pcfg, linear_pair_kernel<false, true>, tmW, tmA, tmB, tmSG, lb) != cudaSuccess)
+  if (cudaLaunchKernelEx(&pcfg, linear_pair_kernel<false, true>, tmW, tmAb, tmB, tmSG, lb) != cudaSuccess)
     return DORA_ERR_CUDA;
 
   // 3) s^2 H = s (s c B)^T B, then dA = [(s c B)^T | s^2 H] [W ; A]
@@ -940,7 +963,8 @@ int dora_factored_norm_bwd(const void* W, const void* A, const void* B, float s,
   la.kb_main = static_cast<int>(cdiv(d_out, kLinBK));
   la.kb_total = la.kb_main + static_cast<int>(cdiv(r, kLinBK));
   la.tiles_m = static_cast<int>(cdiv(r, kPairBM));
-  la.tiles_n = static_cast<int>(cdiv(d_in, kPairBN));
+  la.bn = bn_a;
+  la.tiles_n = static_cast<int>(cdiv(d_in, bn_a));
   la.stages = stages;
   la.stage_bytes = kPairStageBytes;
   la.alpha = 1.f;

@@ -52,6 +52,7 @@ struct LinearArgs {
   int M, N;                // output rows and columns
   int kb_main, kb_total;   // K blocks from the first operand pair; total with the extension pair
   int tiles_m, tiles_n;
+  int bn;                  // pair tile width along N: 128, 192 or 256 (each CTA holds bn / 2)
   int stages;
   uint32_t stage_bytes;
   float alpha;             // uniform scale of the product
@@ -129,6 +130,12 @@ __global__ void __launch_bounds__(kLinThreads, 1)
   const int n_pairs = gridDim.x >> 1;
   const long long limit = a.wait_limit;
   const int n_tiles = a.tiles_m * a.tiles_n;
+  const int half_bn = a.bn / 2;
+  // MN-major B: 64-column boxes per K block covering this CTA's bn / 2 columns
+  const int mn_boxes = (half_bn + 63) / 64;
+  // bytes one CTA's copies bring per stage
+  const uint32_t stage_tx =
+      kPairKps * (kLinABytes + (B_MN ? static_cast<uint32_t>(mn_boxes) * (kLinABytes / 2) : half_bn * 128u));
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.stages; ++s) {
@@ -174,7 +181,7 @@ __global__ void __launch_bounds__(kLinThreads, 1)
       int tm, tn;
       lin_tile(a, t, tm, tn);
       const int ya = tm * kPairBM + static_cast<int>(rank) * kLinBM;
-      const int yb = tn * kPairBN + static_cast<int>(rank) * (kPairBN / 2);
+      const int yb = tn * a.bn + static_cast<int>(rank) * (a.bn / 2);
       for (int kb0 = 0; kb0 < a.kb_total; kb0 += kPairKps) {
         // K blocks past kb_total load boxes that lie wholly outside the
         // tensor: zero-filled, they add nothing
@@ -186,7 +193,7 @@ __global__ void __launch_bounds__(kLinThreads, 1)
         bool got = true;
         if (lane == 0) {
           got = mbar_wait(&empty[stage], phase ^ 1u, limit);
-          if (got && leader) mbar_arrive_expect_tx(&full[stage], 2 * kPairStageBytes);
+          if (got && leader) mbar_arrive_expect_tx(&full[stage], 2 * stage_tx);
           if (!got) lin_timeout(a.status, abort_flag);
         }
         got = __shfl_sync(0xffffffffu, got, 0);
@@ -208,9 +215,9 @@ __global__ void __launch_bounds__(kLinThreads, 1)
           const bool ext = kb >= a.kb_main && a.kb_total > a.kb_main;
           const int xk = (ext ? kb - a.kb_main : kb) * kLinBK;
           tma_load_2d_pair(dst + (kPairKps + i) * kLinABytes, ext ? &tmB2 : &tmB1, bar, xk, yb);
-        } else if (B_MN && lane < 3 * kPairKps) {
-          // K block i: columns yb.. and yb + 64.. of rows (K) kb * 64 .., two 8 KB boxes
-          const int i = (lane - kPairKps) >> 1, h = (lane - kPairKps) & 1;
+        } else if (B_MN && lane < kPairKps + kPairKps * mn_boxes) {
+          // K block i: columns yb + 64 h .. of rows (K) kb * 64 .., 8 KB boxes
+          const int i = (lane - kPairKps) / mn_boxes, h = (lane - kPairKps) % mn_boxes;
           const int kb = kb0 + i;
           const bool ext = kb >= a.kb_main && a.kb_total > a.kb_main;
           const int yk = (ext ? kb - a.kb_main : kb) * kLinBK;
@@ -236,7 +243,7 @@ __global__ void __launch_bounds__(kLinThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      const uint32_t idesc = idesc_bf16_f32(kPairBM, kPairBN) | (B_MN ? kIdescBMnMajor : 0u);
+      const uint32_t idesc = idesc_bf16_f32(kPairBM, a.bn) | (B_MN ? kIdescBMnMajor : 0u);
       const uint64_t desc0 = sw128_kmajor_desc(base_s);
       const uint64_t desc_step = kPairStageBytes >> 4;
       // MN-major B: the two 64-column boxes of a K block are 8 KB apart (the
@@ -298,8 +305,8 @@ __global__ void __launch_bounds__(kLinThreads, 1)
       const bool row_ok = row < a.M;
       const float rscale = (row_ok && a.rs_num) ? __ldg(a.rs_num + row) / __ldg(a.rs_den + row) : 1.f;
 #pragma unroll 1
-      for (int c = 0; c < kPairBN / 32; ++c) {
-        const int col0 = tn * kPairBN + c * 32;
+      for (int c = 0; c < a.bn / 32; ++c) {
+        const int col0 = tn * a.bn + c * 32;
         if (col0 >= a.N) break;  // warp-uniform
         float v[32];
         tmem_ld32(tmem_lane + static_cast<uint32_t>(ab * kPairBN + c * 32), v);
