@@ -215,8 +215,9 @@ def run_ours(args, rank, world, local_rank):
     dense = run_dense_comparator(D, dev, W, A, B, s, ws_n) if rank == 0 else None
     batched = run_batched_context(D, dev) if rank == 0 else None
     fused = run_fused_linear_context(D, dev, wl, W, A, B, m, n) if rank == 0 else None
+    norm_bwd = run_norm_backward_context(D, dev, wl, W, A, B, n) if rank == 0 else None
     return dict(t_total=t_total, t_norm=t_norm, t_fwd=t_fwd, t_bwd=t_bwd, clocks=clocks, status=status, e2e=e2e,
-                wl=wl, dense=dense, batched=batched, fused=fused)
+                wl=wl, dense=dense, batched=batched, fused=fused, norm_bwd=norm_bwd)
 
 
 def run_dense_comparator(D, dev, W, A, B, s, ws_n, reps=10):
@@ -304,6 +305,56 @@ def run_fused_linear_context(D, dev, wl, W, A, B, m, n, reps=10):
                     "bias: dora_fused_linear_fwd vs cuBLAS GEMMs + dora_compose_fwd; context only",
             "fused_us": t_f * 1e6, "unfused_us": t_u * 1e6, "flops": F, "fused_tflops": F / t_f / 1e12,
             "speedup_vs_unfused": t_u / t_f, "gpu_launches_per_call": 2, "device_status": D.dora_device_status()}
+
+
+def norm_backward_flops(d_out, d_in, r):
+    """Algorithmic FLOPs of the attached-norm backward: dB = s c * ([W | B] [A | sG]^T)
+    and dA = [(s c B)^T | s^2 H] [W ; A], plus G = A A^T and H = (c B)^T B."""
+    return 4.0 * d_out * r * (d_in + r) + 2.0 * r * r * (d_in + d_out)
+
+
+def run_norm_backward_context(D, dev, wl, W, A, B, n, reps=10):
+    """Gradients of the row norms into A and B (norm kept attached):
+    dora_factored_norm_bwd against torch.autograd through the dense
+    ||W + s B A||_row (bf16 product, fp32 norm) that frameworks would run.
+    Context beside the step, CUDA events."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(2468)
+    d_n = torch.randn(wl.d_out, generator=g, device=dev)
+    dA = torch.empty(wl.r, wl.d_in, device=dev)
+    dB = torch.empty(wl.d_out, wl.r, device=dev)
+    ws = torch.empty(D.dora_factored_norm_bwd_workspace_size(wl.d_out, wl.d_in, wl.r), dtype=torch.uint8, device=dev)
+    Ab = A.detach().clone().requires_grad_()
+    Bb = B.detach().clone().requires_grad_()
+
+    def factored():
+        D.dora_factored_norm_bwd(W, A, B, wl.s, n, d_n, dA=dA, dB=dB, workspace=ws)
+
+    def dense():
+        Ab.grad = None
+        Bb.grad = None
+        torch.linalg.vector_norm((W + wl.s * (Bb @ Ab)).float(), dim=1).backward(d_n)
+
+    def timed(f):
+        for _ in range(3):
+            f()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            f()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps * 1e-3
+
+    t_f = timed(factored)
+    t_d = timed(dense)
+    F = norm_backward_flops(wl.d_out, wl.d_in, wl.r)
+    return {"what": f"dL/dA, dL/dB through n = ||W + sBA||_row at {wl.d_out} x {wl.d_in}, r = {wl.r}, bf16: "
+                    "dora_factored_norm_bwd vs torch.autograd of the dense norm; context only",
+            "factored_us": t_f * 1e6, "dense_us": t_d * 1e6, "flops": F, "factored_tflops": F / t_f / 1e12,
+            "speedup_vs_dense": t_d / t_f, "workspace_bytes": ws.numel(), "gpu_launches_per_call": 6,
+            "device_status": D.dora_device_status()}
 
 
 # the seven adapted projections of one decoder block of an 8B-class model
@@ -558,6 +609,12 @@ def build_line(args, res, N, peaks, peak_src, traffic, cpu):
         line["dense_comparator"] = res["dense"]
     if res.get("batched") is not None:
         line["many_modules"] = res["batched"]
+    if res.get("norm_bwd"):
+        nb = dict(res["norm_bwd"])
+        nb["frac"] = nb["factored_tflops"] / peaks["bf16_tflops"]
+        nb["peak"] = peaks["bf16_tflops"]
+        nb["bound"] = "tensor"
+        line["norm_backward"] = nb
     if res.get("fused"):
         fl = dict(res["fused"])
         # ten calls back to back (~8 ms): between the burst and the sustained
