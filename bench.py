@@ -151,12 +151,18 @@ def max_over_ranks(values, world, device):
     return t.tolist()
 
 
+def workload_of(args):
+    wl = WL.WORKLOADS[args.workload]
+    tokens = getattr(args, "tokens", None)
+    return wl.with_(tokens=tokens) if tokens else wl
+
+
 def run_ours(args, rank, world, local_rank):
     from factored_weight_norm_b200 import dora as D
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    wl = WL.WORKLOADS[args.workload]
+    wl = workload_of(args)
     T, d_out, d_in, r, s = wl.tokens, wl.d_out, wl.d_in, wl.r, wl.s
     W, A, B, m = WL.make_weights(wl, dev)
     _, base, lora = WL.make_activations(wl, W, A, B, dev)
@@ -212,10 +218,11 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- end to end through the Python API with pinned host buffers
     e2e = run_e2e(args, D, dev, wl, W, A, B, m, base, lora, dy, n, y, d_base, d_lora, d_m, ws_n, ws_b, world)
-    dense = run_dense_comparator(D, dev, W, A, B, s, ws_n) if rank == 0 else None
-    batched = run_batched_context(D, dev) if rank == 0 else None
-    fused = run_fused_linear_context(D, dev, wl, W, A, B, m, n) if rank == 0 else None
-    norm_bwd = run_norm_backward_context(D, dev, wl, W, A, B, n) if rank == 0 else None
+    ctx = rank == 0 and not getattr(args, "no_context", False)
+    dense = run_dense_comparator(D, dev, W, A, B, s, ws_n) if ctx else None
+    batched = run_batched_context(D, dev) if ctx else None
+    fused = run_fused_linear_context(D, dev, wl, W, A, B, m, n) if ctx else None
+    norm_bwd = run_norm_backward_context(D, dev, wl, W, A, B, n) if ctx else None
     return dict(t_total=t_total, t_norm=t_norm, t_fwd=t_fwd, t_bwd=t_bwd, clocks=clocks, status=status, e2e=e2e,
                 wl=wl, dense=dense, batched=batched, fused=fused, norm_bwd=norm_bwd)
 
@@ -503,7 +510,7 @@ def time_oracle(wl, norm_rows, compose_tokens, seed=0):
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
-    wl = WL.WORKLOADS[args.workload]
+    wl = workload_of(args)
     for _ in range(args.warmup):
         time_oracle(wl, *ORACLE_SAMPLE)
     res = []
@@ -637,6 +644,11 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WL.HEADLINE.name, choices=sorted(WL.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed CPU oracle sample")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the workload's token count (compose and fused-linear activations)")
+    ap.add_argument("--no-context", action="store_true",
+                    help="skip the context measurements after the timed step (dense comparator, many modules, "
+                         "fused linear, attached-norm backward), e.g. for a profiler's launch list")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
