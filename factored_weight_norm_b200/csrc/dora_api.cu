@@ -263,8 +263,9 @@ int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_
   ga.wait_limit = kWaitLimitCycles;
   ga.partial = Gp;
   ga.status = dev->status;
+  ga.n_ctas1 = p.gram_tiles * ga.splits;
   const size_t gram_smem = kGramStages * kGramStageBytes + (2 * kGramStages + 1) * 8 + 16 + 1024;
-  gram_tc_kernel<<<p.gram_tiles * ga.splits, kNormThreads, gram_smem, st>>>(tmA, tmA, ga);
+  gram_tc_kernel<<<p.gram_tiles * ga.splits, kNormThreads, gram_smem, st>>>(tmA, tmA, tmA, tmA, ga);
   if (launch_error()) return DORA_ERR_CUDA;
 
   cudaLaunchAttribute pdl[1];
@@ -276,11 +277,14 @@ int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_
   cfg.numAttrs = 1;
 
   const long long rr = static_cast<long long>(r) * r;
-  cfg.gridDim = dim3(static_cast<unsigned>(std::max<long long>(cdiv(p.m_tiles, 256), std::min<long long>(cdiv(rr, 1024), 4 * dev->num_sms))));
+  const unsigned red_grid = static_cast<unsigned>(
+      std::max<long long>(cdiv(p.m_tiles, 256), std::min<long long>(cdiv(rr, 1024), 4 * dev->num_sms)));
+  cfg.gridDim = dim3(red_grid);
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = 0;
   if (cudaLaunchKernelEx(&cfg, gram_reduce_kernel, static_cast<const float*>(Gp), ga.splits, static_cast<int>(r),
-                         0.5f * s, Gs, cnt, p.m_tiles) != cudaSuccess)
+                         0.5f * s, Gs, cnt, p.m_tiles, static_cast<int>(red_grid), static_cast<const float*>(nullptr), 0,
+                         0.f, static_cast<__nv_bfloat16*>(nullptr)) != cudaSuccess)
     return DORA_ERR_CUDA;
 
   NormArgs na{};
@@ -806,16 +810,19 @@ int dora_fused_linear_fwd(const void* x, const void* W, const void* A, const voi
 // ---------------------------------------------------- attached-norm backward
 namespace {
 struct BwdLayout {
-  int nt, splits_max;
-  size_t off_part, off_sg, off_h, off_bt, off_bct, total;
+  int nt, splits_max;  // K splits of each of the two Gram products (G and H) in one launch
+  size_t off_part, off_part2, off_sg, off_h, off_bt, off_bct, total;
 };
 BwdLayout bwd_layout(int64_t d_out, int64_t r) {
   BwdLayout L{};
   L.nt = static_cast<int>(cdiv(r, kBoxRows));
-  L.splits_max = std::max(1, std::min(kMaxGramSplits, 160 / (L.nt * L.nt)));
+  L.splits_max = std::max(1, std::min(kMaxGramSplits, 80 / (L.nt * L.nt)));
+  const size_t part_bytes = static_cast<size_t>(L.splits_max) * L.nt * L.nt * kBoxRows * kBoxRows * 4;
   size_t off = 0;
   L.off_part = off;
-  off = align_up(off + static_cast<size_t>(L.splits_max) * L.nt * L.nt * kBoxRows * kBoxRows * 4, 256);
+  off = align_up(off + part_bytes, 256);
+  L.off_part2 = off;
+  off = align_up(off + part_bytes, 256);
   L.off_sg = off;
   off = align_up(off + static_cast<size_t>(r) * r * 2, 256);
   L.off_h = off;
@@ -862,6 +869,7 @@ int dora_factored_norm_bwd(const void* W, const void* A, const void* B, float s,
   if (device_info(&dev)) return DORA_ERR_CUDA;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* part = reinterpret_cast<float*>(ws + L.off_part);
+  float* part2 = reinterpret_cast<float*>(ws + L.off_part2);
   __nv_bfloat16* sG = reinterpret_cast<__nv_bfloat16*>(ws + L.off_sg);
   __nv_bfloat16* s2H = reinterpret_cast<__nv_bfloat16*>(ws + L.off_h);
   __nv_bfloat16* Bt = reinterpret_cast<__nv_bfloat16*>(ws + L.off_bt);
@@ -884,33 +892,40 @@ int dora_factored_norm_bwd(const void* W, const void* A, const void* B, float s,
   cudaLaunchAttribute pdl[1];
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
+
+  // 2) one Gram launch for both products: G = A A^T over d_in and
+  //    s H = (s c B)^T B over d_out (split-K partial tiles), then one fixed-order
+  //    reduction writing bf16 s G and s^2 H
+  const int kb_g = static_cast<int>(cdiv(d_in, kBK)), kb_h = static_cast<int>(cdiv(d_out, kBK));
+  GramArgs ga{};
+  ga.r = static_cast<int>(r);
+  ga.n_tiles = L.nt;
+  ga.kb_main = kb_g;
+  ga.splits = std::max(1, std::min({L.splits_max, (dev->num_sms / 2) / (L.nt * L.nt), kb_g}));
+  ga.kb_main2 = kb_h;
+  ga.splits2 = std::max(1, std::min({L.splits_max, (dev->num_sms / 2) / (L.nt * L.nt), kb_h}));
+  ga.n_ctas1 = L.nt * L.nt * ga.splits;
+  ga.partial = part;
+  ga.partial2 = part2;
+  ga.wait_limit = kWaitLimitCycles;
+  ga.status = dev->status;
   const size_t gram_smem = kGramStages * kGramStageBytes + (2 * kGramStages + 1) * 8 + 16 + 1024;
-  // split-K Gram-type product M-side x N-side^T (r x r) over kb K blocks, then
-  // the fixed-order reduction scaled by `scale` into bf16 `out`
-  auto gram_pair = [&](const CUtensorMap& mside, const CUtensorMap& nside, int kb, float scale,
-                       __nv_bfloat16* out) -> int {
-    GramArgs ga{};
-    ga.r = static_cast<int>(r);
-    ga.kb_main = kb;
-    ga.n_tiles = L.nt;
-    ga.splits = std::max(1, std::min({L.splits_max, dev->num_sms / (L.nt * L.nt), kb}));
-    ga.wait_limit = kWaitLimitCycles;
-    ga.partial = part;
-    ga.status = dev->status;
-    gram_tc_kernel<<<L.nt * L.nt * ga.splits, kNormThreads, gram_smem, st>>>(mside, nside, ga);
-    if (launch_error()) return DORA_ERR_CUDA;
+  gram_tc_kernel<<<ga.n_ctas1 + L.nt * L.nt * ga.splits2, kNormThreads, gram_smem, st>>>(tmA, tmA, tmBct, tmBt, ga);
+  if (launch_error()) return DORA_ERR_CUDA;
+  {
     cudaLaunchConfig_t cfg{};
     cfg.stream = st;
     cfg.attrs = pdl;
     cfg.numAttrs = 1;
     const long long rr = static_cast<long long>(r) * r;
-    cfg.gridDim = dim3(static_cast<unsigned>(std::max<long long>(1, std::min<long long>(cdiv(rr, 1024), 4 * dev->num_sms))));
+    const int g1 = static_cast<int>(std::max<long long>(1, std::min<long long>(cdiv(rr, 1024), 2 * dev->num_sms)));
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * g1));
     cfg.blockDim = dim3(256);
-    if (cudaLaunchKernelEx(&cfg, gram_reduce_kernel, static_cast<const float*>(part), ga.splits, static_cast<int>(r),
-                           scale, out, static_cast<int*>(nullptr), 0) != cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, gram_reduce_kernel, static_cast<const float*>(part), ga.splits, static_cast<int>(r), s,
+                           sG, static_cast<int*>(nullptr), 0, g1, static_cast<const float*>(part2), ga.splits2, s,
+                           s2H) != cudaSuccess)
       return DORA_ERR_CUDA;
-    return DORA_OK;
-  };
+  }
 
   cudaLaunchAttribute attrs[2];
   attrs[0].id = cudaLaunchAttributeClusterDimension;
@@ -931,8 +946,8 @@ int dora_factored_norm_bwd(const void* W, const void* A, const void* B, float s,
                                                               static_cast<long long>(la.tiles_m) * la.tiles_n)));
   };
 
-  // 2) s G, then dB = s c * ([W | B] [A | s G]^T)
-  if (int e = gram_pair(tmA, tmA, static_cast<int>(cdiv(d_in, kBK)), s, sG)) return e;
+  // 3) dB = s c * ([W | B] [A | s G]^T), waiting for the reduction only
+  //    before its K-extension blocks
   LinearArgs lb{};
   lb.M = static_cast<int>(d_out);
   lb.N = static_cast<int>(r);
@@ -955,8 +970,10 @@ int dora_factored_norm_bwd(const void* W, const void* A, const void* B, float s,
   if (cudaLaunchKernelEx(&pcfg, linear_pair_kernel<false, true>, tmW, tmAb, tmB, tmSG, lb) != cudaSuccess)
     return DORA_ERR_CUDA;
 
-  // 3) s^2 H = s (s c B)^T B, then dA = [(s c B)^T | s^2 H] [W ; A]
-  if (int e = gram_pair(tmBct, tmBt, static_cast<int>(cdiv(d_out, kBK)), s, s2H)) return e;
+  // 4) dA = [(s c B)^T | s^2 H] [W ; A], dependent on dB through programmatic
+  //    dependent launch: its CTAs take the SMs dB leaves free or finishes
+  //    with; before its extension blocks it waits for dB's completion, which
+  //    follows the reduction's
   LinearArgs la{};
   la.M = static_cast<int>(r);
   la.N = static_cast<int>(d_in);

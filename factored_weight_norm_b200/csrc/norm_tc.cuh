@@ -503,6 +503,11 @@ struct GramArgs {
   long long wait_limit;
   float* partial;  // [splits][n_tiles^2][128][128] fp32
   int* status;
+  // optional second product of the same r x r shape in the same launch:
+  // CTAs from n_ctas1 on compute it from the second pair of maps
+  int n_ctas1;     // CTAs of the first product (= the grid when there is no second)
+  int kb_main2, splits2;
+  float* partial2;
 };
 
 constexpr int kGramKPerStage = 2;  // K blocks per ring stage: 4 boxes, one per producer lane
@@ -510,7 +515,8 @@ constexpr int kGramStages = 3;
 constexpr uint32_t kGramStageBytes = 2 * kGramKPerStage * kBoxBytes;
 
 __global__ void __launch_bounds__(kNormThreads, 1)
-    gram_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const GramArgs a) {
+    gram_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2, const GramArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   const uint32_t base_s = (raw_s + 1023u) & ~1023u;
@@ -525,15 +531,23 @@ __global__ void __launch_bounds__(kNormThreads, 1)
   const int lane = threadIdx.x & 31;
   const long long limit = a.wait_limit;
 
-  // (tile, K split) of this CTA; every tile of the n_tiles x n_tiles grid is
-  // computed so the reduction reads each output element contiguously
-  const int split = blockIdx.x % a.splits;
-  const int tile = blockIdx.x / a.splits;
+  // which product, then (tile, K split) of this CTA; every tile of the
+  // n_tiles x n_tiles grid is computed so the reduction reads each output
+  // element contiguously
+  const bool second = static_cast<int>(blockIdx.x) >= a.n_ctas1;
+  const int bid = second ? static_cast<int>(blockIdx.x) - a.n_ctas1 : static_cast<int>(blockIdx.x);
+  const int splits = second ? a.splits2 : a.splits;
+  const int kb_main = second ? a.kb_main2 : a.kb_main;
+  float* const partial = second ? a.partial2 : a.partial;
+  const CUtensorMap* const mapM = second ? &tmA2 : &tmA;
+  const CUtensorMap* const mapN = second ? &tmB2 : &tmB;
+  const int split = bid % splits;
+  const int tile = bid / splits;
   const int mi = tile / a.n_tiles;
   const int ni = tile % a.n_tiles;
   const int n_this = min(kBoxRows, a.r - ni * kBoxRows);
-  const int kb_lo = static_cast<int>(static_cast<long long>(split) * a.kb_main / a.splits);
-  const int kb_hi = static_cast<int>(static_cast<long long>(split + 1) * a.kb_main / a.splits);
+  const int kb_lo = static_cast<int>(static_cast<long long>(split) * kb_main / splits);
+  const int kb_hi = static_cast<int>(static_cast<long long>(split + 1) * kb_main / splits);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kGramStages; ++s) {
@@ -545,8 +559,8 @@ __global__ void __launch_bounds__(kNormThreads, 1)
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(mapM);
+    tma_prefetch_desc(mapN);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 128);
@@ -574,7 +588,7 @@ __global__ void __launch_bounds__(kNormThreads, 1)
       if (!__shfl_sync(0xffffffffu, got, 0)) break;
       __syncwarp();
       if (lane < 2 * nk)
-        tma_load_2d(base_s + stage * kGramStageBytes + lane * kBoxBytes, (lane & 1) ? &tmB : &tmA, &full[stage],
+        tma_load_2d(base_s + stage * kGramStageBytes + lane * kBoxBytes, (lane & 1) ? mapN : mapM, &full[stage],
                     (kb0 + (lane >> 1)) * kBK, ((lane & 1) ? ni : mi) * kBoxRows);
       parity_bits = (parity_bits & ~(1u << stage)) | (phase << stage);
       filled_mask |= 1u << stage;
@@ -619,7 +633,7 @@ __global__ void __launch_bounds__(kNormThreads, 1)
     const bool ok = mbar_wait_warp(tmem_full, 0, limit);
     if (ok && !__any_sync(0xffffffffu, *abort_flag != 0)) {
       tc_fence_after();
-      float* dst = a.partial + (static_cast<size_t>(split) * a.n_tiles * a.n_tiles + tile) * (kBoxRows * kBoxRows) +
+      float* dst = partial + (static_cast<size_t>(split) * a.n_tiles * a.n_tiles + tile) * (kBoxRows * kBoxRows) +
                    static_cast<size_t>(row_local) * kBoxRows;
       for (int j0 = 0; j0 < n_this; j0 += 32) {
         float acc[32];
@@ -644,19 +658,31 @@ __global__ void __launch_bounds__(kNormThreads, 1)
 
 // Sums the K splits of G = A A^T in fixed order, scales by s/2 and writes the
 // bf16 G' the norm kernel's K extension reads; also zeroes the norm kernel's
-// tile counters.
+// tile counters.  CTAs from `g1` on reduce a second product the same way
+// (`partial2`, `splits2`, `scale2`, `Gs2`; a Gram launch of two products).
 __global__ void gram_reduce_kernel(const float* __restrict__ partial, int splits, int r, float half_s,
-                                   __nv_bfloat16* __restrict__ Gs, int* counters, int n_counters) {
+                                   __nv_bfloat16* __restrict__ Gs, int* counters, int n_counters, int g1,
+                                   const float* __restrict__ partial2, int splits2, float scale2,
+                                   __nv_bfloat16* __restrict__ Gs2) {
   grid_dep_launch();
   grid_dep_wait();  // the Gram partial tiles are complete
+  if (static_cast<int>(blockIdx.x) >= g1) {
+    partial = partial2;
+    splits = splits2;
+    half_s = scale2;
+    Gs = Gs2;
+    n_counters = 0;
+  }
+  const int bx = static_cast<int>(blockIdx.x) >= g1 ? static_cast<int>(blockIdx.x) - g1 : static_cast<int>(blockIdx.x);
+  const int gx = static_cast<int>(blockIdx.x) >= g1 ? static_cast<int>(gridDim.x) - g1 : g1;
   const long long total = static_cast<long long>(r) * r;
   const int nt = (r + kBoxRows - 1) / kBoxRows;
   const long long split_stride = static_cast<long long>(nt) * nt * kBoxRows * kBoxRows;
   // four elements per thread and eight splits per round: 32 independent loads
   // in flight; each element still adds its splits in increasing order
   constexpr int kE = 4, kS = 8;
-  const long long step = static_cast<long long>(gridDim.x) * blockDim.x;
-  for (long long base = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; base < total;
+  const long long step = static_cast<long long>(gx) * blockDim.x;
+  for (long long base = bx * static_cast<long long>(blockDim.x) + threadIdx.x; base < total;
        base += kE * step) {
     long long src[kE];
     float sum[kE];
@@ -684,7 +710,7 @@ __global__ void gram_reduce_kernel(const float* __restrict__ partial, int splits
     for (int e = 0; e < kE; ++e)
       if (base + e * step < total) Gs[base + e * step] = __float2bfloat16_rn(half_s * sum[e]);
   }
-  const int tid = blockIdx.x * blockDim.x + threadIdx.x;
+  const int tid = bx * static_cast<int>(blockDim.x) + static_cast<int>(threadIdx.x);
   if (tid < n_counters) counters[tid] = 0;
 }
 
