@@ -123,3 +123,19 @@ def test_fused_linear_workspace_reuse_and_errors():
         D.dora_fused_linear_fwd(x, W, A, B, m, n, s, workspace=ws[:100])
     with pytest.raises(TypeError):
         D.dora_fused_linear_fwd(x.float(), W, A, B, m, n, s)
+
+
+def test_fused_linear_mlp_up_shape_sampled():
+    # the largest configured projection: 16384 tokens x (5120 -> 27648), r = 384
+    wl = wlmod.MLP_UP_32B
+    W, A, B, m = wlmod.make_weights(wl, DEV)
+    g = torch.Generator(device=DEV).manual_seed(9)
+    x = torch.randn(wl.tokens, wl.d_in, generator=g, device=DEV).to(torch.bfloat16)
+    n = D.dora_factored_norm(W, A, B, wl.s)
+    y = D.dora_fused_linear_fwd(x, W, A, B, m.float().contiguous(), n, wl.s)
+    torch.cuda.synchronize()
+    assert D.dora_device_status() == D.DORA_OK
+    rows = np.array([0, 255, 256, 9999, 16383])
+    cols = np.array([0, 191, 192, 13824, 27647])
+    ref = _ref(x, W, A, B, None, m, n, wl.s, rows=rows, cols=cols)
+    P.assert_act_close(P.f64(y)[rows][:, cols], ref, "y sampled")

@@ -108,3 +108,22 @@ def test_norm_bwd_degenerate_sizes_and_determinism():
     D.dora_factored_norm_bwd(W[:0], A, B[:0], 0.5, n[:0], d_n[:0], dA=dA)
     torch.cuda.synchronize()
     assert not dA.any()
+
+
+def test_norm_bwd_mlp_up_shape_sampled():
+    # the largest configured projection: 27648 x 5120, r = 384
+    wl = wlmod.MLP_UP_32B
+    W, A, B, _ = wlmod.make_weights(wl, DEV)
+    n = D.dora_factored_norm(W, A, B, wl.s)
+    g = torch.Generator(device=DEV).manual_seed(4)
+    d_n = torch.randn(wl.d_out, generator=g, device=DEV)
+    dA, dB = D.dora_factored_norm_bwd(W, A, B, wl.s, n, d_n)
+    torch.cuda.synchronize()
+    assert D.dora_device_status() == D.DORA_OK
+    W64, A64, B64, n64, dn64 = P.f64(W), P.f64(A), P.f64(B), P.f64(n), P.f64(d_n)
+    rows = np.array([0, 255, 13824, 27647])
+    _, rB = oracle.norm_backward(W64[rows], A64, B64[rows], wl.s, n64[rows], dn64[rows])
+    assert_grad_close(P.f64(dB)[rows], rB, "dB rows")
+    cols = np.array([0, 255, 256, 5119])
+    rA, _ = oracle.norm_backward(W64[:, cols], A64[:, cols], B64, wl.s, n64, dn64)
+    assert_grad_close(P.f64(dA)[:, cols], rA, "dA columns")
