@@ -511,8 +511,14 @@ int dora_factored_norm(const void* W, const void* A, const void* B, int64_t d_ou
   return launch_error();
 }
 
-int dora_compose_fwd(const void* base_out, const void* lora_out, const void* bias, const float* m, const float* n,
-                     float s, int64_t tokens, int64_t d_out, dora_dtype dt, void* y, void* stream) {
+int dora_compose_fwd(const void* base_out, const void* lora_out, const float* m, const float* n, float s,
+                     int64_t tokens, int64_t d_out, dora_dtype dt, void* y, void* stream) {
+  return dora_compose_fwd_bias(base_out, lora_out, nullptr, m, n, s, tokens, d_out, dt, y, stream);
+}
+
+int dora_compose_fwd_bias(const void* base_out, const void* lora_out, const void* bias, const float* m,
+                          const float* n, float s, int64_t tokens, int64_t d_out, dora_dtype dt, void* y,
+                          void* stream) {
   if (dt != DORA_BF16 && dt != DORA_F32) return DORA_ERR_UNSUPPORTED;
   if (tokens < 0 || d_out < 0) return DORA_ERR_INVALID_ARG;
   if (tokens == 0 || d_out == 0) return DORA_OK;
@@ -564,9 +570,17 @@ size_t dora_compose_bwd_workspace_size(int64_t tokens, int64_t d_out) {
   return align_up(strips * 4, 256) + align_up(static_cast<size_t>(kMaxBwdChunks) * std::max<int64_t>(d_out, 1) * 4, 256);
 }
 
-int dora_compose_bwd(const void* dy, const void* base_out, const void* lora_out, const void* bias, const float* m,
-                     const float* n, float s, int64_t tokens, int64_t d_out, dora_dtype dt, void* d_base, void* d_lora,
-                     float* d_m, void* workspace, size_t workspace_bytes, void* stream) {
+int dora_compose_bwd(const void* dy, const void* base_out, const void* lora_out, const float* m, const float* n,
+                     float s, int64_t tokens, int64_t d_out, dora_dtype dt, void* d_base, void* d_lora, float* d_m,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  return dora_compose_bwd_bias(dy, base_out, lora_out, nullptr, m, n, s, tokens, d_out, dt, d_base, d_lora, d_m,
+                               workspace, workspace_bytes, stream);
+}
+
+int dora_compose_bwd_bias(const void* dy, const void* base_out, const void* lora_out, const void* bias,
+                          const float* m, const float* n, float s, int64_t tokens, int64_t d_out, dora_dtype dt,
+                          void* d_base, void* d_lora, float* d_m, void* workspace, size_t workspace_bytes,
+                          void* stream) {
   if (dt != DORA_BF16 && dt != DORA_F32) return DORA_ERR_UNSUPPORTED;
   if (tokens < 0 || d_out < 0) return DORA_ERR_INVALID_ARG;
   if (d_out == 0) return DORA_OK;
@@ -1035,9 +1049,17 @@ int noalloc_scratch(unsigned char** out) {
 }  // namespace
 }  // namespace dora
 
-extern "C" int dora_compose_bwd_noalloc(const void* dy, const void* base_out, const void* lora_out, const void* bias,
-                                        const float* m, const float* n, float s, int64_t tokens, int64_t d_out,
-                                        dora_dtype dt, void* d_base, void* d_lora, float* d_m, void* stream) {
+extern "C" int dora_compose_bwd_noalloc(const void* dy, const void* base_out, const void* lora_out, const float* m,
+                                        const float* n, float s, int64_t tokens, int64_t d_out, dora_dtype dt,
+                                        void* d_base, void* d_lora, float* d_m, void* stream) {
+  return dora_compose_bwd_noalloc_bias(dy, base_out, lora_out, nullptr, m, n, s, tokens, d_out, dt, d_base, d_lora,
+                                       d_m, stream);
+}
+
+extern "C" int dora_compose_bwd_noalloc_bias(const void* dy, const void* base_out, const void* lora_out,
+                                             const void* bias, const float* m, const float* n, float s,
+                                             int64_t tokens, int64_t d_out, dora_dtype dt, void* d_base,
+                                             void* d_lora, float* d_m, void* stream) {
   if (dt != DORA_BF16 && dt != DORA_F32) return DORA_ERR_UNSUPPORTED;
   if (tokens < 0 || d_out < 0) return DORA_ERR_INVALID_ARG;
   if (d_out > DORA_NOALLOC_MAX_D_OUT) return DORA_ERR_UNSUPPORTED;

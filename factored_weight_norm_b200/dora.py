@@ -48,15 +48,29 @@ SIGNATURES = {
     ),
     "dora_compose_fwd": (
         ctypes.c_int,
+        [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _f32, _i64, _i64, ctypes.c_int, _c_void_p, _c_void_p],
+    ),
+    "dora_compose_fwd_bias": (
+        ctypes.c_int,
         [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _f32, _i64, _i64, ctypes.c_int, _c_void_p, _c_void_p],
     ),
     "dora_compose_bwd_workspace_size": (_size, [_i64, _i64]),
     "dora_compose_bwd": (
         ctypes.c_int,
+        [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _f32, _i64, _i64, ctypes.c_int,
+         _c_void_p, _c_void_p, _c_void_p, _c_void_p, _size, _c_void_p],
+    ),
+    "dora_compose_bwd_bias": (
+        ctypes.c_int,
         [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _f32, _i64, _i64, ctypes.c_int,
          _c_void_p, _c_void_p, _c_void_p, _c_void_p, _size, _c_void_p],
     ),
     "dora_compose_bwd_noalloc": (
+        ctypes.c_int,
+        [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _f32, _i64, _i64, ctypes.c_int,
+         _c_void_p, _c_void_p, _c_void_p, _c_void_p],
+    ),
+    "dora_compose_bwd_noalloc_bias": (
         ctypes.c_int,
         [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _f32, _i64, _i64, ctypes.c_int,
          _c_void_p, _c_void_p, _c_void_p, _c_void_p],
@@ -258,10 +272,12 @@ def dora_compose_fwd(base_out, lora_out, m, n, s: float, y=None, stream=None, bi
     _check_bias(bias, base_out, "dora_compose_fwd")
     if y is None:
         y = torch.empty_like(base_out)
-    st = lib().dora_compose_fwd(
-        _ptr(base_out), _ptr(lora_out), _ptr(bias), _ptr(m), _ptr(n), float(s), tokens, d_out, _dt(base_out), _ptr(y),
-        _stream(stream),
-    )
+    head = (_ptr(base_out), _ptr(lora_out))
+    tail = (_ptr(m), _ptr(n), float(s), tokens, d_out, _dt(base_out), _ptr(y), _stream(stream))
+    if bias is None:
+        st = lib().dora_compose_fwd(*head, *tail)
+    else:
+        st = lib().dora_compose_fwd_bias(*head, _ptr(bias), *tail)
     _check(st, "dora_compose_fwd")
     return y
 
@@ -285,11 +301,13 @@ def dora_compose_bwd(dy, base_out, lora_out, m, n, s: float, d_base=None, d_lora
     need = dora_compose_bwd_workspace_size(tokens, d_out)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=base_out.device)
-    st = lib().dora_compose_bwd(
-        _ptr(dy), _ptr(base_out), _ptr(lora_out), _ptr(bias), _ptr(m), _ptr(n), float(s), tokens, d_out,
-        _dt(base_out), _ptr(d_base), _ptr(d_lora), _ptr(d_m), _ptr(workspace),
-        workspace.numel() * workspace.element_size(), _stream(stream),
-    )
+    head = (_ptr(dy), _ptr(base_out), _ptr(lora_out))
+    tail = (_ptr(m), _ptr(n), float(s), tokens, d_out, _dt(base_out), _ptr(d_base), _ptr(d_lora), _ptr(d_m),
+            _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    if bias is None:
+        st = lib().dora_compose_bwd(*head, *tail)
+    else:
+        st = lib().dora_compose_bwd_bias(*head, _ptr(bias), *tail)
     _check(st, "dora_compose_bwd")
     return d_base, d_lora, d_m
 
@@ -306,10 +324,13 @@ def dora_compose_bwd_noalloc(dy, base_out, lora_out, m, n, s: float, d_base, d_l
     if m.dtype != torch.float32 or n.dtype != torch.float32 or d_m.dtype != torch.float32:
         raise TypeError("m, n and d_m must be fp32")
     _check_bias(bias, base_out, "dora_compose_bwd_noalloc")
-    st = lib().dora_compose_bwd_noalloc(
-        _ptr(dy), _ptr(base_out), _ptr(lora_out), _ptr(bias), _ptr(m), _ptr(n), float(s), tokens, d_out,
-        _dt(base_out), _ptr(d_base), _ptr(d_lora), _ptr(d_m), _stream(stream),
-    )
+    head = (_ptr(dy), _ptr(base_out), _ptr(lora_out))
+    tail = (_ptr(m), _ptr(n), float(s), tokens, d_out, _dt(base_out), _ptr(d_base), _ptr(d_lora), _ptr(d_m),
+            _stream(stream))
+    if bias is None:
+        st = lib().dora_compose_bwd_noalloc(*head, *tail)
+    else:
+        st = lib().dora_compose_bwd_noalloc_bias(*head, _ptr(bias), *tail)
     _check(st, "dora_compose_bwd_noalloc")
     return d_base, d_lora, d_m
 

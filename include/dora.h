@@ -114,43 +114,54 @@ DORA_API int dora_factored_norm_batched(const dora_norm_problem* problems, int c
  * composition collapsed into a single pass, in a numerically stable form for
  * the near-unity regime):
  *
- *   g = m / n,  delta = (m - n) / n                  (fp32, per output channel)
- *   y = base + (delta * (base - b) + g * s * lora)   (fp32 arithmetic, one rounding)
+ *   g = m / n,  delta = (m - n) / n            (fp32, per output channel)
+ *   y = base + (delta * base + g * s * lora)   (fp32 arithmetic, one rounding)
  *
- * which equals b + g * ((base - b) + s * lora) without rounding g or g - 1 to
- * the activation type.
+ * which equals g * (base + s * lora) without rounding g or g - 1 to the
+ * activation type.  base_out, lora_out, y: [tokens, d_out] row-major in dt
+ * (bf16: d_out a multiple of 8 and 16-byte aligned pointers; fp32: 4-byte
+ * aligned); lora_out is the unscaled (x A^T) B^T.  m, n: fp32 [d_out] (n from
+ * dora_factored_norm).  tokens may be 0 (nothing is launched).  y must not
+ * overlap the inputs. */
+DORA_API int dora_compose_fwd(const void* base_out, const void* lora_out, const float* m, const float* n, float s,
+                              int64_t tokens, int64_t d_out, dora_dtype dt, void* y, void* stream);
+
+/* dora_compose_fwd for a base layer with a bias b:
  *
- * base_out, lora_out, y: [tokens, d_out] row-major in dt (bf16: d_out a
- * multiple of 8 and 16-byte aligned pointers; fp32: 4-byte aligned).
- * base_out is the frozen base layer's output x W^T + b, lora_out the unscaled
- * (x A^T) B^T.  bias: the base layer's b, [d_out] in dt (bf16: 16-byte
- * aligned; fp32: 4-byte aligned), or NULL for a layer without one (b = 0,
- * bit-identical to the no-bias form).  The pages never
- * mention a bias; the rescaling is taken to act on the weight's product only,
- * as the DoRA summary page's Method defines the adapted weight m V / ||V||.
- * m, n: fp32 [d_out] (n from dora_factored_norm).  tokens may be 0 (nothing
- * is launched).  y must not overlap the inputs. */
-DORA_API int dora_compose_fwd(const void* base_out, const void* lora_out, const void* bias, const float* m,
-                              const float* n, float s, int64_t tokens, int64_t d_out, dora_dtype dt, void* y,
-                              void* stream);
+ *   y = base + (delta * (base - b) + g * s * lora) = b + g * ((base - b) + s * lora)
+ *
+ * base_out is the frozen base layer's output x W^T + b.  bias: [d_out] in dt
+ * (bf16: 16-byte aligned; fp32: 4-byte aligned), or NULL, which is exactly
+ * dora_compose_fwd.  The pages never mention a bias; the rescaling is taken to
+ * act on the weight's product only, as the DoRA summary page's Method defines
+ * the adapted weight m V / ||V||. */
+DORA_API int dora_compose_fwd_bias(const void* base_out, const void* lora_out, const void* bias, const float* m,
+                                   const float* n, float s, int64_t tokens, int64_t d_out, dora_dtype dt, void* y,
+                                   void* stream);
 
 /* Bytes of workspace dora_compose_bwd needs (column partial sums). */
 DORA_API size_t dora_compose_bwd_workspace_size(int64_t tokens, int64_t d_out);
 
-/* Backward of dora_compose_fwd with n held constant (the norm is detached)
- * and the bias frozen (no gradient is returned for it):
+/* Backward of dora_compose_fwd with n held constant (the norm is detached):
  *
  *   d_base = g * dy,   d_lora = s * g * dy,
- *   d_m_i  = (sum_t dy[t,i] * ((base[t,i] - b_i) + s * lora[t,i])) / n_i
+ *   d_m_i  = (sum_t dy[t,i] * (base[t,i] + s * lora[t,i])) / n_i
  *
- * bias as in dora_compose_fwd (NULL: b = 0).
  * d_base, d_lora: [tokens, d_out] in dt, overwritten.  d_m: fp32 [d_out],
  * overwritten (tokens == 0 gives d_m = 0).  The token reduction accumulates
  * in fp32 and combines per-chunk partials in a fixed order. */
-DORA_API int dora_compose_bwd(const void* dy, const void* base_out, const void* lora_out, const void* bias,
-                              const float* m, const float* n, float s, int64_t tokens, int64_t d_out, dora_dtype dt,
-                              void* d_base, void* d_lora, float* d_m, void* workspace, size_t workspace_bytes,
-                              void* stream);
+DORA_API int dora_compose_bwd(const void* dy, const void* base_out, const void* lora_out, const float* m,
+                              const float* n, float s, int64_t tokens, int64_t d_out, dora_dtype dt, void* d_base,
+                              void* d_lora, float* d_m, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward of dora_compose_fwd_bias (bias frozen, no gradient returned for it):
+ * as dora_compose_bwd with d_m_i = (sum_t dy[t,i] * ((base[t,i] - b_i) +
+ * s * lora[t,i])) / n_i.  bias as in dora_compose_fwd_bias; NULL is exactly
+ * dora_compose_bwd. */
+DORA_API int dora_compose_bwd_bias(const void* dy, const void* base_out, const void* lora_out, const void* bias,
+                                   const float* m, const float* n, float s, int64_t tokens, int64_t d_out,
+                                   dora_dtype dt, void* d_base, void* d_lora, float* d_m, void* workspace,
+                                   size_t workspace_bytes, void* stream);
 
 /* Largest d_out dora_compose_bwd_noalloc accepts, and the size of the
  * library-owned scratch array behind it (8 KiB of counters + 16 row chunks of
@@ -178,9 +189,17 @@ DORA_API int dora_compose_bwd(const void* dy, const void* base_out, const void* 
  * example on two streams without ordering between them) race and give wrong
  * results; order them on one stream.  d_out > DORA_NOALLOC_MAX_D_OUT returns
  * DORA_ERR_UNSUPPORTED and launches nothing. */
-DORA_API int dora_compose_bwd_noalloc(const void* dy, const void* base_out, const void* lora_out, const void* bias,
-                                      const float* m, const float* n, float s, int64_t tokens, int64_t d_out,
-                                      dora_dtype dt, void* d_base, void* d_lora, float* d_m, void* stream);
+DORA_API int dora_compose_bwd_noalloc(const void* dy, const void* base_out, const void* lora_out, const float* m,
+                                      const float* n, float s, int64_t tokens, int64_t d_out, dora_dtype dt,
+                                      void* d_base, void* d_lora, float* d_m, void* stream);
+
+/* dora_compose_bwd_bias with the library-owned scratch of
+ * dora_compose_bwd_noalloc (same rules); NULL bias is exactly
+ * dora_compose_bwd_noalloc. */
+DORA_API int dora_compose_bwd_noalloc_bias(const void* dy, const void* base_out, const void* lora_out,
+                                           const void* bias, const float* m, const float* n, float s, int64_t tokens,
+                                           int64_t d_out, dora_dtype dt, void* d_base, void* d_lora, float* d_m,
+                                           void* stream);
 
 /* Bytes of workspace dora_factored_norm_bwd needs: O(r^2 + r d_out), no
  * d_out x d_in term (the Gram partial tiles, s G and s^2 H in bf16, and two

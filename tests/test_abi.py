@@ -121,35 +121,48 @@ def test_batched_workspace_has_no_dense_term(lib):
 
 def test_compose_argument_errors(lib):
     f = lib.dora_compose_fwd
+    assert f(None, FAKE, FAKE, FAKE, 0.5, 4, 64, D.DORA_BF16, FAKE, None) == D.DORA_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, FAKE, 0.5, -1, 64, D.DORA_BF16, FAKE, None) == D.DORA_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, FAKE, 0.5, 4, 60, D.DORA_BF16, FAKE, None) == D.DORA_ERR_UNSUPPORTED
+    assert f(FAKE, MISALIGNED, FAKE, FAKE, 0.5, 4, 64, D.DORA_BF16, FAKE, None) == D.DORA_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, FAKE, 0.5, 0, 64, D.DORA_BF16, FAKE, None) == D.DORA_OK
+    b = lib.dora_compose_bwd
+    ws = lib.dora_compose_bwd_workspace_size(4, 64)
+    # dy, base, lora, m, n, s, tokens, d_out, dt, d_base, d_lora, d_m, workspace, bytes, stream
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, 0.5, 4, 64, D.DORA_BF16, FAKE, FAKE, FAKE, FAKE, ws, None]
+    bad = list(args)
+    bad[11] = None  # d_m
+    assert b(*bad) == D.DORA_ERR_INVALID_ARG
+    bad = list(args)
+    bad[13] = ws - 1
+    assert b(*bad) == D.DORA_ERR_WORKSPACE
+    bad = list(args)
+    bad[12] = None
+    assert b(*bad) == D.DORA_ERR_WORKSPACE
+    bad = list(args)
+    bad[7] = 12
+    assert b(*bad) == D.DORA_ERR_UNSUPPORTED
+
+
+def test_compose_bias_argument_errors(lib):
     odd = ctypes.c_void_p(0x10001)
-    assert f(None, FAKE, None, FAKE, FAKE, 0.5, 4, 64, D.DORA_BF16, FAKE, None) == D.DORA_ERR_INVALID_ARG
-    assert f(FAKE, FAKE, None, FAKE, FAKE, 0.5, -1, 64, D.DORA_BF16, FAKE, None) == D.DORA_ERR_INVALID_ARG
-    assert f(FAKE, FAKE, None, FAKE, FAKE, 0.5, 4, 60, D.DORA_BF16, FAKE, None) == D.DORA_ERR_UNSUPPORTED
-    assert f(FAKE, MISALIGNED, None, FAKE, FAKE, 0.5, 4, 64, D.DORA_BF16, FAKE, None) == D.DORA_ERR_UNSUPPORTED
+    f = lib.dora_compose_fwd_bias
+    # base, lora, bias, m, n, s, tokens, d_out, dt, y, stream
+    assert f(None, FAKE, FAKE, FAKE, FAKE, 0.5, 4, 64, D.DORA_BF16, FAKE, None) == D.DORA_ERR_INVALID_ARG
     assert f(FAKE, FAKE, odd, FAKE, FAKE, 0.5, 4, 64, D.DORA_BF16, FAKE, None) == D.DORA_ERR_UNSUPPORTED
     assert f(FAKE, FAKE, MISALIGNED, FAKE, FAKE, 0.5, 4, 64, D.DORA_BF16, FAKE, None) == D.DORA_ERR_UNSUPPORTED
     assert f(FAKE, FAKE, MISALIGNED, FAKE, FAKE, 0.5, 4, 64, D.DORA_F32, FAKE, None) == D.DORA_ERR_UNSUPPORTED
-    assert f(FAKE, FAKE, None, FAKE, FAKE, 0.5, 0, 64, D.DORA_BF16, FAKE, None) == D.DORA_OK
-    b = lib.dora_compose_bwd
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 0.5, 0, 64, D.DORA_BF16, FAKE, None) == D.DORA_OK
+    b = lib.dora_compose_bwd_bias
     ws = lib.dora_compose_bwd_workspace_size(4, 64)
-    # dy, base, lora, bias, m, n, s, tokens, d_out, dt, d_base, d_lora, d_m, workspace, bytes, stream
-    args = [FAKE, FAKE, FAKE, None, FAKE, FAKE, 0.5, 4, 64, D.DORA_BF16, FAKE, FAKE, FAKE, FAKE, ws, None]
-    bad = list(args)
-    bad[12] = None  # d_m
-    assert b(*bad) == D.DORA_ERR_INVALID_ARG
-    bad = list(args)
-    bad[14] = ws - 1
-    assert b(*bad) == D.DORA_ERR_WORKSPACE
-    bad = list(args)
-    bad[13] = None
-    assert b(*bad) == D.DORA_ERR_WORKSPACE
-    bad = list(args)
-    bad[8] = 12
-    assert b(*bad) == D.DORA_ERR_UNSUPPORTED
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0.5, 4, 64, D.DORA_BF16, FAKE, FAKE, FAKE, FAKE, ws, None]
     bad = list(args)
     bad[3] = MISALIGNED  # a bf16 bias must be 16-byte aligned
     assert b(*bad) == D.DORA_ERR_UNSUPPORTED
-    na = lib.dora_compose_bwd_noalloc
+    bad = list(args)
+    bad[12] = None  # d_m
+    assert b(*bad) == D.DORA_ERR_INVALID_ARG
+    na = lib.dora_compose_bwd_noalloc_bias
     assert na(FAKE, FAKE, FAKE, odd, FAKE, FAKE, 0.5, 4, 64, D.DORA_BF16, FAKE, FAKE, FAKE, None) == D.DORA_ERR_UNSUPPORTED
     assert na(FAKE, FAKE, FAKE, None, FAKE, FAKE, 0.5, 4, 64, D.DORA_BF16, FAKE, FAKE, None, None) == D.DORA_ERR_INVALID_ARG
 

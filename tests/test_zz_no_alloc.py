@@ -37,7 +37,7 @@ def _noalloc(dy, base, lora, m, n, s, d_base, d_lora, d_m):
     d_lora.fill_(float("nan"))
     d_m.fill_(float("nan"))
     st = D.lib().dora_compose_bwd_noalloc(
-        _ptr(dy), _ptr(base), _ptr(lora), None, _ptr(m), _ptr(n), s, T, d_out,
+        _ptr(dy), _ptr(base), _ptr(lora), _ptr(m), _ptr(n), s, T, d_out,
         D.DORA_BF16 if base.dtype == torch.bfloat16 else D.DORA_F32,
         _ptr(d_base), _ptr(d_lora), _ptr(d_m), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == D.DORA_OK, D.status_string(st)
@@ -63,6 +63,6 @@ def test_noalloc_matches_workspace_version_twice(T, d_out, dtype):
 
 def test_noalloc_rejects_d_out_above_its_maximum():
     fake = ctypes.c_void_p(0x10000)
-    st = D.lib().dora_compose_bwd_noalloc(fake, fake, fake, None, fake, fake, 0.5, 4, MAX_D_OUT + 8, D.DORA_BF16,
+    st = D.lib().dora_compose_bwd_noalloc(fake, fake, fake, fake, fake, 0.5, 4, MAX_D_OUT + 8, D.DORA_BF16,
                                           fake, fake, fake, None)
     assert st == D.DORA_ERR_UNSUPPORTED
