@@ -219,10 +219,17 @@ def run_ours(args, rank, world, local_rank):
     # ---- end to end through the Python API with pinned host buffers
     e2e = run_e2e(args, D, dev, wl, W, A, B, m, base, lora, dy, n, y, d_base, d_lora, d_m, ws_n, ws_b, world)
     ctx = rank == 0 and not getattr(args, "no_context", False)
-    dense = run_dense_comparator(D, dev, W, A, B, s, ws_n) if ctx else None
-    batched = run_batched_context(D, dev) if ctx else None
-    fused = run_fused_linear_context(D, dev, wl, W, A, B, m, n) if ctx else None
-    norm_bwd = run_norm_backward_context(D, dev, wl, W, A, B, n) if ctx else None
+    # each context measurement starts from an idle GPU (a short host pause),
+    # and the power-hungry fused-linear GEMMs run last
+    def idle_then(f):
+        torch.cuda.synchronize()
+        time.sleep(0.25)
+        return f()
+
+    dense = idle_then(lambda: run_dense_comparator(D, dev, W, A, B, s, ws_n)) if ctx else None
+    batched = idle_then(lambda: run_batched_context(D, dev)) if ctx else None
+    norm_bwd = idle_then(lambda: run_norm_backward_context(D, dev, wl, W, A, B, n)) if ctx else None
+    fused = idle_then(lambda: run_fused_linear_context(D, dev, wl, W, A, B, m, n)) if ctx else None
     return dict(t_total=t_total, t_norm=t_norm, t_fwd=t_fwd, t_bwd=t_bwd, clocks=clocks, status=status, e2e=e2e,
                 wl=wl, dense=dense, batched=batched, fused=fused, norm_bwd=norm_bwd)
 
@@ -360,7 +367,7 @@ def run_norm_backward_context(D, dev, wl, W, A, B, n, reps=10):
     return {"what": f"dL/dA, dL/dB through n = ||W + sBA||_row at {wl.d_out} x {wl.d_in}, r = {wl.r}, bf16: "
                     "dora_factored_norm_bwd vs torch.autograd of the dense norm; context only",
             "factored_us": t_f * 1e6, "dense_us": t_d * 1e6, "flops": F, "factored_tflops": F / t_f / 1e12,
-            "speedup_vs_dense": t_d / t_f, "workspace_bytes": ws.numel(), "gpu_launches_per_call": 6,
+            "speedup_vs_dense": t_d / t_f, "workspace_bytes": ws.numel(), "gpu_launches_per_call": 5,
             "device_status": D.dora_device_status()}
 
 
