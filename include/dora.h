@@ -228,7 +228,8 @@ DORA_API size_t dora_factored_norm_bwd_workspace_size(int64_t d_out, int64_t d_i
  * gets none.  r = 0 does nothing; d_out = 0 zeroes dA; d_in = 0 zeroes dB.
  * workspace: at least dora_factored_norm_bwd_workspace_size() bytes,
  * 256-byte aligned, contents ignored.  Only DORA_BF16.  Asynchronous on
- * `stream` (six launches). */
+ * `stream` (five launches: the prep copies, one Gram launch for G and H, its
+ * reduction, the dB and the dA GEMMs). */
 DORA_API int dora_factored_norm_bwd(const void* W, const void* A, const void* B, float s, const float* n,
                                     const float* d_n, int64_t d_out, int64_t d_in, int64_t r, dora_dtype dt,
                                     float* dA, float* dB, void* workspace, size_t workspace_bytes, void* stream);
