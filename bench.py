@@ -70,13 +70,23 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_digest():
+# the sources that define each measured kernel family's code and launches
+TRAFFIC_SOURCES = {
+    "norm": ("sm100_ptx.cuh", "norm_tc.cuh", "dora_api.cu"),
+    "compose_fwd": ("sm100_ptx.cuh", "compose.cuh", "dora_api.cu"),
+    "compose_bwd": ("sm100_ptx.cuh", "compose.cuh", "dora_api.cu"),
+}
+
+
+def source_digest(names=None):
+    """sha256 prefix of the listed csrc files (all .cu/.cuh files by default)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "factored_weight_norm_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(f.read())
+    if names is None:
+        names = [n for n in os.listdir(csrc) if n.endswith((".cu", ".cuh"))]
+    for name in sorted(names):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -87,11 +97,11 @@ def load_traffic():
     out = {}
     if not os.path.exists(p):
         return out
-    digest = source_digest()
     for line in open(p):
         parts = line.split()
-        if len(parts) >= 4 and not line.startswith("#") and parts[1] == digest:
-            out[parts[0]] = {"bytes": float(parts[2]), "workload": parts[3]}
+        if len(parts) >= 4 and not line.startswith("#") and parts[0] in TRAFFIC_SOURCES:
+            if parts[1] == source_digest(TRAFFIC_SOURCES[parts[0]]):
+                out[parts[0]] = {"bytes": float(parts[2]), "workload": parts[3]}
     return out
 
 
