@@ -898,8 +898,8 @@ int dora_factored_norm_bwd(const void* W, const void* A, const void* B, float s,
     return DORA_ERR_CUDA;
 
   // 1) B^T and (s c B)^T
-  norm_bwd_prep_kernel<<<dim3(static_cast<unsigned>(cdiv(d_out, 32)), static_cast<unsigned>(cdiv(r, 32))), 256, 0,
-                         st>>>(static_cast<const __nv_bfloat16*>(B), d_n, n, s, static_cast<int>(d_out),
+  norm_bwd_prep_kernel<<<dim3(static_cast<unsigned>(cdiv(d_out, kPrepTile)), static_cast<unsigned>(cdiv(r, kPrepTile))),
+                         256, 0, st>>>(static_cast<const __nv_bfloat16*>(B), d_n, n, s, static_cast<int>(d_out),
                                static_cast<int>(r), Bt, Bct);
   if (launch_error()) return DORA_ERR_CUDA;
 
