@@ -168,8 +168,8 @@ __global__ void __launch_bounds__(kBwdThreads, 2) compose_bwd_kernel(
     const T* __restrict__ dy, const T* __restrict__ base, const T* __restrict__ lora, const T* __restrict__ bias,
     const float* __restrict__ m,
     const float* __restrict__ n, float s, long long tokens, long long nvec, long long d_out, T* __restrict__ d_base,
-    T* __restrict__ d_lora, float* __restrict__ partial, int* __restrict__ counters, float* __restrict__ d_m,
-    long long rows_per_chunk) {
+    T* __restrict__ d_lora, float* __restrict__ partial, unsigned long long* __restrict__ counters,
+    float* __restrict__ d_m, long long rows_per_chunk, unsigned long long epoch) {
   __shared__ float red[kBwdThreads / 32][kBwdVecs][VEC];
   __shared__ int is_last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -274,7 +274,23 @@ __global__ void __launch_bounds__(kBwdThreads, 2) compose_bwd_kernel(
   }
   __threadfence();
   __syncthreads();
-  if (t == 0) is_last = (atomicAdd(&counters[blockIdx.x], 1) == static_cast<int>(gridDim.y) - 1);
+  // arrivals per column strip in a word tagged with this call's epoch,
+  // (epoch << 8) | count: a word with any other tag (an earlier call, or
+  // whatever the caller's buffer held) counts as zero, so the counters need
+  // no clearing before the launch
+  const unsigned long long tag = epoch << 8;
+  if (t == 0) {
+    unsigned long long* c = counters + blockIdx.x;
+    unsigned long long v = *reinterpret_cast<volatile unsigned long long*>(c);
+    int seen = 0;
+    while (true) {
+      seen = (v & ~0xffull) == tag ? static_cast<int>(v & 0xffull) : 0;
+      const unsigned long long prev = atomicCAS(c, v, tag | static_cast<unsigned long long>(seen + 1));
+      if (prev == v) break;
+      v = prev;
+    }
+    is_last = (seen == static_cast<int>(gridDim.y) - 1);
+  }
   __syncthreads();
   if (is_last) {
     __threadfence();
@@ -283,7 +299,7 @@ __global__ void __launch_bounds__(kBwdThreads, 2) compose_bwd_kernel(
       for (unsigned c = 0; c < gridDim.y; ++c) total += ld_cg_f32(&partial[c * d_out + tcol]);
       d_m[tcol] = total / __ldg(n + tcol);
     }
-    if (t == 0) counters[blockIdx.x] = 0;
+    if (t == 0) counters[blockIdx.x] = tag;  // count 0 under this tag: a replay of the same launch starts clean
   }
 }
 

@@ -12,6 +12,8 @@
 #include <cstdint>
 #include <cstring>
 #include <vector>
+#include <atomic>
+#include <chrono>
 #include <mutex>
 
 #include "../../include/dora.h"
@@ -159,16 +161,25 @@ int make_map(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols, ui
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // One compose backward launch; the bias picks the instantiation.
+// Tag of one compose-backward launch for its arrival counters (56 bits, new
+// for every call in this process; the start mixes in the clock so that a
+// buffer left by another process is unlikely to carry a live tag).
+unsigned long long next_bwd_epoch() {
+  static std::atomic<unsigned long long> counter{
+      static_cast<unsigned long long>(std::chrono::steady_clock::now().time_since_epoch().count()) * 0x9E3779B97F4A7C15ull};
+  return counter.fetch_add(1) & ((1ull << 56) - 1);
+}
+
 template <typename T, int VEC>
 void launch_compose_bwd(dim3 grid, cudaStream_t st, const void* dy, const void* base_out, const void* lora_out,
                         const void* bias, const float* m, const float* n, float s, long long tokens, long long nvec,
-                        long long d_out, void* d_base, void* d_lora, float* part, int* cnt, float* d_m,
+                        long long d_out, void* d_base, void* d_lora, float* part, unsigned long long* cnt, float* d_m,
                         long long rows) {
   auto kernel = bias ? compose_bwd_kernel<T, VEC, true> : compose_bwd_kernel<T, VEC, false>;
   kernel<<<grid, kBwdThreads, 0, st>>>(static_cast<const T*>(dy), static_cast<const T*>(base_out),
                                        static_cast<const T*>(lora_out), static_cast<const T*>(bias), m, n, s, tokens,
                                        nvec, d_out, static_cast<T*>(d_base), static_cast<T*>(d_lora), part, cnt, d_m,
-                                       rows);
+                                       rows, next_bwd_epoch());
 }
 
 // ------------------------------------------------------------ norm planning
@@ -567,7 +578,7 @@ int dora_compose_fwd_bias(const void* base_out, const void* lora_out, const void
 size_t dora_compose_bwd_workspace_size(int64_t tokens, int64_t d_out) {
   if (tokens < 0 || d_out < 0) return 0;
   const size_t strips = static_cast<size_t>(cdiv(std::max<int64_t>(d_out, 1), dora::kBwdVecs));
-  return align_up(strips * 4, 256) + align_up(static_cast<size_t>(kMaxBwdChunks) * std::max<int64_t>(d_out, 1) * 4, 256);
+  return align_up(strips * 8, 256) + align_up(static_cast<size_t>(kMaxBwdChunks) * std::max<int64_t>(d_out, 1) * 4, 256);
 }
 
 int dora_compose_bwd(const void* dy, const void* base_out, const void* lora_out, const float* m, const float* n,
@@ -627,10 +638,9 @@ int dora_compose_bwd_bias(const void* dy, const void* base_out, const void* lora
   const long long rows = cdiv(tokens, chunks);
   const long long chunks2 = cdiv(tokens, rows);
   uint8_t* w = static_cast<uint8_t*>(workspace);
-  int* cnt = reinterpret_cast<int*>(w);
+  unsigned long long* cnt = reinterpret_cast<unsigned long long*>(w);  // tagged: no clearing needed
   const size_t strips_all = static_cast<size_t>(cdiv(d_out, kBwdVecs));
-  float* part = reinterpret_cast<float*>(w + align_up(strips_all * 4, 256));
-  if (cudaMemsetAsync(cnt, 0, static_cast<size_t>(strips) * 4, st) != cudaSuccess) return DORA_ERR_CUDA;
+  float* part = reinterpret_cast<float*>(w + align_up(strips_all * 8, 256));
   dim3 grid(static_cast<unsigned>(strips), static_cast<unsigned>(chunks2));
   if (dt == DORA_BF16)
     launch_compose_bwd<__nv_bfloat16, 8>(grid, st, dy, base_out, lora_out, bias, m, n, s, tokens, nvec, d_out, d_base,
@@ -1021,7 +1031,11 @@ namespace dora {
 namespace {
 
 constexpr int kNoallocChunks = 16;     // row chunks of column partials
-constexpr size_t kNoallocCounterBytes = 8192;
+constexpr size_t kNoallocCounterBytes = 16384;
+// 64-bit tagged arrival counters, one per 16-vector column strip; the most
+// strips come with 1-element vectors at the largest d_out
+static_assert((DORA_NOALLOC_MAX_D_OUT + kBwdVecs - 1) / kBwdVecs * 8 <= kNoallocCounterBytes,
+              "counter area too small for the largest d_out");
 static_assert(DORA_NOALLOC_SCRATCH_BYTES == kNoallocCounterBytes + kNoallocChunks * 4ull * DORA_NOALLOC_MAX_D_OUT,
               "scratch layout and the header's size disagree");
 
@@ -1103,10 +1117,10 @@ extern "C" int dora_compose_bwd_noalloc_bias(const void* dy, const void* base_ou
                                        std::min<long long>(kNoallocChunks, cdiv(tokens, kBwdSlots)));
   const long long rows = cdiv(tokens, chunks);
   const long long chunks2 = cdiv(tokens, rows);
-  int* cnt = reinterpret_cast<int*>(scratch);
+  // tagged strip counters (no clearing needed); the partials are written before read
+  if (static_cast<size_t>(strips) * 8 > kNoallocCounterBytes) return DORA_ERR_UNSUPPORTED;
+  unsigned long long* cnt = reinterpret_cast<unsigned long long*>(scratch);
   float* part = reinterpret_cast<float*>(scratch + kNoallocCounterBytes);
-  // the strip counters must start at zero; the partials are written before read
-  if (cudaMemsetAsync(cnt, 0, static_cast<size_t>(strips) * 4, st) != cudaSuccess) return DORA_ERR_CUDA;
   dim3 grid(static_cast<unsigned>(strips), static_cast<unsigned>(chunks2));
   if (dt == DORA_BF16)
     launch_compose_bwd<__nv_bfloat16, 8>(grid, st, dy, base_out, lora_out, bias, m, n, s, tokens, nvec, d_out, d_base,

@@ -164,10 +164,10 @@ DORA_API int dora_compose_bwd_bias(const void* dy, const void* base_out, const v
                                    size_t workspace_bytes, void* stream);
 
 /* Largest d_out dora_compose_bwd_noalloc accepts, and the size of the
- * library-owned scratch array behind it (8 KiB of counters + 16 row chunks of
+ * library-owned scratch array behind it (16 KiB of counters + 16 row chunks of
  * fp32 column partials). */
 #define DORA_NOALLOC_MAX_D_OUT 32768
-#define DORA_NOALLOC_SCRATCH_BYTES (8192 + 16 * 4 * DORA_NOALLOC_MAX_D_OUT)
+#define DORA_NOALLOC_SCRATCH_BYTES (16384 + 16 * 4 * DORA_NOALLOC_MAX_D_OUT)
 
 /* dora_compose_bwd for callers that cannot allocate device memory at call
  * time and so cannot provide a workspace: code recorded into a CUDA graph or
@@ -183,8 +183,9 @@ DORA_API int dora_compose_bwd_bias(const void* dy, const void* base_out, const v
  * cudaMalloc, cudaFree or allocating library routine is called.  The first
  * call on a device looks the array's device address up (cudaGetSymbolAddress)
  * with that device current; make that first call before any stream capture.
- * Each call clears the counters it needs (cudaMemsetAsync on the array) and
- * the array otherwise keeps the last call's contents.  All calls on a device
+ * Nothing is cleared before a call either: the arrival counters in the array
+ * carry a per-call tag, so whatever they hold is ignored, and the array
+ * keeps the last call's contents.  All calls on a device
  * share the one array, so calls whose executions overlap on the GPU (for
  * example on two streams without ordering between them) race and give wrong
  * results; order them on one stream.  d_out > DORA_NOALLOC_MAX_D_OUT returns

@@ -369,3 +369,19 @@ def test_norm_then_compose_end_to_end(name):
 def test_device_status_clean_after_suite():
     torch.cuda.synchronize()
     assert D.dora_device_status() == D.DORA_OK
+
+
+@pytest.mark.parametrize("fill", [0x00, 0xFF, 0x5A])
+def test_compose_bwd_ignores_workspace_contents(fill):
+    # the column-strip arrival counters carry a per-call tag: whatever the
+    # workspace holds on entry, the result is the one a fresh buffer gives
+    wl = _wl(1024, 64, 16, s=0.5, tokens=777)
+    base, lora, m, n, dy = _compose_inputs(wl)
+    clean = torch.zeros(D.dora_compose_bwd_workspace_size(wl.tokens, wl.d_out), dtype=torch.uint8, device=DEV)
+    ref = [t.clone() for t in D.dora_compose_bwd(dy, base, lora, m, n, wl.s, workspace=clean)]
+    dirty = torch.full_like(clean, fill)
+    for _ in range(2):
+        got = D.dora_compose_bwd(dy, base, lora, m, n, wl.s, workspace=dirty)
+        torch.cuda.synchronize()
+        for a, b in zip(got, ref):
+            assert torch.equal(a, b)

@@ -66,3 +66,16 @@ def test_noalloc_rejects_d_out_above_its_maximum():
     st = D.lib().dora_compose_bwd_noalloc(fake, fake, fake, fake, fake, 0.5, 4, MAX_D_OUT + 8, D.DORA_BF16,
                                           fake, fake, fake, None)
     assert st == D.DORA_ERR_UNSUPPORTED
+
+
+def test_noalloc_f32_scalar_vectors_at_the_largest_width():
+    # fp32 with d_out not a multiple of 4: one element per vector, the most
+    # column strips (2048) and so the most arrival counters the scratch holds
+    T, d_out = 40, MAX_D_OUT - 2
+    dy, base, lora, m, n, s = _inputs(T, d_out, "f32")
+    ref = D.dora_compose_bwd(dy, base, lora, m, n, s)
+    outs = (torch.empty_like(base), torch.empty_like(base), torch.empty(base.shape[1], device="cuda"))
+    got = _noalloc(dy, base, lora, m, n, s, *outs)
+    torch.cuda.synchronize()
+    for g, r, name in zip(got, ref, ("d_base", "d_lora", "d_m")):
+        P.assert_act_close(g, P.f64(r), name)
