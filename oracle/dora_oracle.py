@@ -36,6 +36,12 @@ upstream gradient ``dy``:
     d_lora = s * g * dy
     d_m_i  = sum_t dy[t, i] * (base[t, i] + s * lora[t, i]) / n_i
 
+Two more definitions serve the paths built on top of these:
+
+    linear_forward:  y = b + g * (x W'^T)           the adapted layer itself
+    norm_backward:   dV = (d_n / n) V', dB = s dV A^T, dA = s B^T dV
+                     (the row norms' gradients into A and B, norm attached)
+
 Layout convention (PyTorch ``nn.Linear``): ``W`` is ``[d_out, d_in]``, ``A``
 (lora_A) is ``[r, d_in]``, ``B`` (lora_B) is ``[d_out, r]``; activations are
 ``[tokens, d_out]`` row-major; ``m``/``n`` are per output channel.  The
