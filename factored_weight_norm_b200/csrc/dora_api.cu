@@ -789,8 +789,7 @@ int dora_fused_linear_fwd(const void* x, const void* W, const void* A, const voi
     pa.bn = bn_p;
     pa.tiles_n = static_cast<int>(cdiv(r, bn_p));
     pa.stages = stages;
-    pa.stage_bytes = kPairStageBytes;
-    pa.alpha = s;
+      pa.alpha = s;
     pa.out = P;
     pa.ldo = r;
     pa.wait_limit = kWaitLimitCycles;
@@ -811,7 +810,6 @@ int dora_fused_linear_fwd(const void* x, const void* W, const void* A, const voi
   la.bn = bn_y;
   la.tiles_n = static_cast<int>(cdiv(d_out, bn_y));
   la.stages = stages;
-  la.stage_bytes = kPairStageBytes;
   la.alpha = 1.f;
   la.m = m;
   la.n = n;
@@ -981,7 +979,6 @@ int dora_factored_norm_bwd(const void* W, const void* A, const void* B, float s,
   lb.bn = bn_b;
   lb.tiles_n = static_cast<int>(cdiv(r, bn_b));
   lb.stages = stages;
-  lb.stage_bytes = kPairStageBytes;
   lb.alpha = s;
   lb.rs_num = d_n;
   lb.rs_den = n;
@@ -1007,7 +1004,6 @@ int dora_factored_norm_bwd(const void* W, const void* A, const void* B, float s,
   la.bn = bn_a;
   la.tiles_n = static_cast<int>(cdiv(d_in, bn_a));
   la.stages = stages;
-  la.stage_bytes = kPairStageBytes;
   la.alpha = 1.f;
   la.out = dA;
   la.ldo = d_in;

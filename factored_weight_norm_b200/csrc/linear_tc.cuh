@@ -53,8 +53,7 @@ struct LinearArgs {
   int kb_main, kb_total;   // K blocks from the first operand pair; total with the extension pair
   int tiles_m, tiles_n;
   int bn;                  // pair tile width along N: 128, 192 or 256 (each CTA holds bn / 2)
-  int stages;
-  uint32_t stage_bytes;
+  int stages;             // ring stages of kPairStageBytes
   float alpha;             // uniform scale of the product
   const float* m;          // per-column g = m / n, or null (g = 1)
   const float* n;
