@@ -139,3 +139,9 @@ def test_fused_linear_mlp_up_shape_sampled():
     cols = np.array([0, 191, 192, 13824, 27647])
     ref = _ref(x, W, A, B, None, m, n, wl.s, rows=rows, cols=cols)
     P.assert_act_close(P.f64(y)[rows][:, cols], ref, "y sampled")
+
+
+def test_fused_linear_no_output_channels():
+    x, W, A, B, b, m, n, s = _case(64, 128, 256, 16)
+    y = D.dora_fused_linear_fwd(x, W[:0].contiguous(), A, B[:0].contiguous(), m[:0], n[:0], s)
+    assert y.shape == (64, 0)

@@ -127,3 +127,24 @@ def test_norm_bwd_mlp_up_shape_sampled():
     cols = np.array([0, 255, 256, 5119])
     rA, _ = oracle.norm_backward(W64[:, cols], A64[:, cols], B64, wl.s, n64, dn64)
     assert_grad_close(P.f64(dA)[:, cols], rA, "dA columns")
+
+
+def test_norm_bwd_no_input_columns_zeroes_dB():
+    # d_in = 0: V = W + sBA is empty per row, n = 0 would be the forward, and
+    # the gradient into B is exactly zero (written, not left as it was)
+    W, A, B, n, d_n = _case(256, 512, 64, 0.5)
+    dB = torch.full((256, 64), 7.0, device=DEV)
+    D.dora_factored_norm_bwd(W[:, :0].contiguous(), A[:, :0].contiguous(), B, 0.5, n, d_n, dB=dB)
+    torch.cuda.synchronize()
+    assert not dB.any()
+
+
+@pytest.mark.parametrize("r", [1024])
+def test_norm_bwd_large_rank(r):
+    W, A, B, n, d_n = _case(512, 1024, r, 0.5)
+    dA, dB = D.dora_factored_norm_bwd(W, A, B, 0.5, n, d_n)
+    torch.cuda.synchronize()
+    assert D.dora_device_status() == D.DORA_OK
+    rA, rB = oracle.norm_backward(P.f64(W), P.f64(A), P.f64(B), 0.5, P.f64(n), P.f64(d_n))
+    assert_grad_close(dA, rA, "dA")
+    assert_grad_close(dB, rB, "dB")

@@ -385,3 +385,16 @@ def test_compose_bwd_ignores_workspace_contents(fill):
         torch.cuda.synchronize()
         for a, b in zip(got, ref):
             assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("shape", [(256, 1024, 4096), (384, 520, 2048)], ids=lambda s: "x".join(map(str, s)))
+def test_norm_bf16_largest_ranks(shape):
+    # the largest accepted rank (4096): 8 N chunks of 512, a 32 x 32 tile Gram,
+    # rank above d_in
+    d_out, d_in, r = shape
+    wl = _wl(d_out, d_in, r, s=0.5)
+    W, A, B, _ = wlmod.make_weights(wl, DEV)
+    n = D.dora_factored_norm(W, A, B, wl.s)
+    torch.cuda.synchronize()
+    assert D.dora_device_status() == D.DORA_OK
+    P.assert_norm_close(n, _oracle_norm(W, A, B, wl.s), torch.bfloat16)
