@@ -249,7 +249,7 @@ long long pick_chunks(long long cols, long long slots, long long k_max) {
 }
 
 int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_t d_in, int64_t r, float s,
-              float* n_out, void* ws, cudaStream_t st, DeviceInfo* dev) {
+              float* n_out, void* ws, cudaStream_t st, DeviceInfo* dev, bool squared) {
   const TcPlan p = plan_tc(d_out, d_in, r);
   uint8_t* w = static_cast<uint8_t*>(ws);
   __nv_bfloat16* Gs = reinterpret_cast<__nv_bfloat16*>(w + p.off_gs);
@@ -321,6 +321,7 @@ int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_
   na.counters = cnt;
   na.n_out = n_out;
   na.status = dev->status;
+  na.squared = squared ? 1 : 0;
   const int grid = static_cast<int>(std::min<long long>({static_cast<long long>(dev->num_sms), p.units, kMaxGrid}));
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kNormThreads);
@@ -464,6 +465,14 @@ int norm_batched(const dora_norm_problem* q, const BatchLayout& L, uint8_t* ws, 
 
 using namespace dora;
 
+namespace dora {
+namespace {
+// The factored norm, n = sqrt(max(n^2, 0)) or, with `squared`, n^2 as summed.
+int factored_norm(const void* W, const void* A, const void* B, int64_t d_out, int64_t d_in, int64_t r, float s,
+                  dora_dtype dt, float* n_out, void* workspace, size_t workspace_bytes, void* stream, bool squared);
+}  // namespace
+}  // namespace dora
+
 extern "C" {
 
 const char* dora_status_string(int status) {
@@ -488,6 +497,32 @@ size_t dora_factored_norm_workspace_size(int64_t d_out, int64_t d_in, int64_t r,
 
 int dora_factored_norm(const void* W, const void* A, const void* B, int64_t d_out, int64_t d_in, int64_t r, float s,
                        dora_dtype dt, float* n_out, void* workspace, size_t workspace_bytes, void* stream) {
+  return factored_norm(W, A, B, d_out, d_in, r, s, dt, n_out, workspace, workspace_bytes, stream, false);
+}
+
+int dora_factored_norm_sq(const void* W, const void* A, const void* B, int64_t d_out, int64_t d_in, int64_t r,
+                          float s, dora_dtype dt, float* n2_out, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  return factored_norm(W, A, B, d_out, d_in, r, s, dt, n2_out, workspace, workspace_bytes, stream, true);
+}
+
+int dora_norm_finish(float* n, int64_t d_out, void* stream) {
+  if (d_out < 0) return DORA_ERR_INVALID_ARG;
+  if (d_out == 0) return DORA_OK;
+  if (!n) return DORA_ERR_INVALID_ARG;
+  if (!aligned(n, 4)) return DORA_ERR_UNSUPPORTED;
+  DeviceInfo* dev = nullptr;
+  if (device_info(&dev)) return DORA_ERR_CUDA;
+  norm_finish_kernel<<<static_cast<unsigned>(cdiv(d_out, 256)), 256, 0, static_cast<cudaStream_t>(stream)>>>(n, d_out);
+  return launch_error();
+}
+
+}  // extern "C"
+
+namespace dora {
+namespace {
+int factored_norm(const void* W, const void* A, const void* B, int64_t d_out, int64_t d_in, int64_t r, float s,
+                  dora_dtype dt, float* n_out, void* workspace, size_t workspace_bytes, void* stream, bool squared) {
   const int arg = norm_arg_status(W, A, B, d_out, d_in, r, dt, n_out);
   if (arg != DORA_OK || d_out == 0) return arg;
   const size_t need = dora_factored_norm_workspace_size(d_out, d_in, r, dt);
@@ -504,13 +539,13 @@ int dora_factored_norm(const void* W, const void* A, const void* B, int64_t d_ou
     const int blocks = static_cast<int>(cdiv(d_out, 8));
     if (dt == DORA_BF16)
       rownorm_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(W), static_cast<int>(d_out),
-                                                            static_cast<int>(d_in), n_out);
+                                                            static_cast<int>(d_in), n_out, squared ? 1 : 0);
     else
       rownorm_kernel<float><<<blocks, 256, 0, st>>>(static_cast<const float*>(W), static_cast<int>(d_out),
-                                                    static_cast<int>(d_in), n_out);
+                                                    static_cast<int>(d_in), n_out, squared ? 1 : 0);
     return launch_error();
   }
-  if (dt == DORA_BF16) return norm_bf16(W, A, B, d_out, d_in, r, s, n_out, workspace, st, dev);
+  if (dt == DORA_BF16) return norm_bf16(W, A, B, d_out, d_in, r, s, n_out, workspace, st, dev, squared);
   float* G = static_cast<float*>(workspace);
   const long long pairs = r * (r + 1) / 2;
   const int gblocks = static_cast<int>(std::min<long long>(cdiv(pairs, 8), 8LL * dev->num_sms));
@@ -518,9 +553,13 @@ int dora_factored_norm(const void* W, const void* A, const void* B, int64_t d_ou
   if (launch_error()) return DORA_ERR_CUDA;
   norm_f32_kernel<<<static_cast<unsigned>(d_out), 256, 0, st>>>(
       static_cast<const float*>(W), static_cast<const float*>(A), static_cast<const float*>(B), G,
-      static_cast<int>(d_out), static_cast<int>(d_in), static_cast<int>(r), s, n_out);
+      static_cast<int>(d_out), static_cast<int>(d_in), static_cast<int>(r), s, n_out, squared ? 1 : 0);
   return launch_error();
 }
+}  // namespace
+}  // namespace dora
+
+extern "C" {
 
 int dora_compose_fwd(const void* base_out, const void* lora_out, const float* m, const float* n, float s,
                      int64_t tokens, int64_t d_out, dora_dtype dt, void* y, void* stream) {

@@ -49,7 +49,7 @@ __global__ void gram_f32_kernel(const float* __restrict__ A, int r, int d_in, fl
 __global__ void __launch_bounds__(256) norm_f32_kernel(const float* __restrict__ W, const float* __restrict__ A,
                                                        const float* __restrict__ B, const float* __restrict__ G,
                                                        int d_out, int d_in, int r, float s,
-                                                       float* __restrict__ n_out) {
+                                                       float* __restrict__ n_out, int squared) {
   __shared__ float red[3][8];
   const int i = blockIdx.x;
   if (i >= d_out) return;
@@ -93,13 +93,13 @@ __global__ void __launch_bounds__(256) norm_f32_kernel(const float* __restrict__
       g += red[2][w];
     }
     const float n2 = b + 2.f * s * x + s * s * g;
-    n_out[i] = sqrtf(fmaxf(n2, 0.f));
+    n_out[i] = squared ? n2 : sqrtf(fmaxf(n2, 0.f));
   }
 }
 
 // Plain row norm ||W_i|| (rank-0 adapter, or s*BA == 0 by construction).
 template <typename T>
-__global__ void rownorm_kernel(const T* __restrict__ W, int d_out, int d_in, float* __restrict__ n_out) {
+__global__ void rownorm_kernel(const T* __restrict__ W, int d_out, int d_in, float* __restrict__ n_out, int squared) {
   const int warps = blockDim.x >> 5;
   const int i = blockIdx.x * warps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -111,7 +111,14 @@ __global__ void rownorm_kernel(const T* __restrict__ W, int d_out, int d_in, flo
     acc = fmaf(v, v, acc);
   }
   acc = warp_sum(acc);
-  if (lane == 0) n_out[i] = sqrtf(acc);
+  if (lane == 0) n_out[i] = squared ? acc : sqrtf(acc);
+}
+
+// n = sqrt(max(n^2, 0)) in place: the last step of a norm whose squared
+// partials were summed across d_in shards.
+__global__ void norm_finish_kernel(float* __restrict__ n, long long d_out) {
+  const long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+  if (i < d_out) n[i] = sqrtf(fmaxf(n[i], 0.f));
 }
 
 }  // namespace dora

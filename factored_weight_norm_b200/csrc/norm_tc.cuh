@@ -55,6 +55,7 @@ struct NormArgs {
   int* counters;          // [m_tiles], zeroed by gram_reduce_kernel
   float* n_out;           // [d_out]
   int* status;
+  int squared;            // 1: write n^2 as summed (a shard's partial), 0: sqrt(max(n^2, 0))
 };
 
 // Owner CTA of unit u when U units are split into G contiguous ranges
@@ -467,7 +468,7 @@ __global__ void __launch_bounds__(kNormThreads, 1)
 #pragma unroll
         for (int j = 0; j < kRows; ++j) {
           const int row2 = x.mt * kBM + lane + 32 * j;
-          if (row2 < a.d_out) a.n_out[row2] = sqrtf(fmaxf(total[j], 0.f));
+          if (row2 < a.d_out) a.n_out[row2] = a.squared ? total[j] : sqrtf(fmaxf(total[j], 0.f));
         }
         if (lane == 0) a.counters[x.mt] = 0;
       }

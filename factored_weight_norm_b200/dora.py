@@ -87,6 +87,11 @@ SIGNATURES = {
         [_c_void_p, _c_void_p, _c_void_p, _f32, _c_void_p, _c_void_p, _i64, _i64, _i64, ctypes.c_int, _c_void_p,
          _c_void_p, _c_void_p, _size, _c_void_p],
     ),
+    "dora_factored_norm_sq": (
+        ctypes.c_int,
+        [_c_void_p, _c_void_p, _c_void_p, _i64, _i64, _i64, _f32, ctypes.c_int, _c_void_p, _c_void_p, _size, _c_void_p],
+    ),
+    "dora_norm_finish": (ctypes.c_int, [_c_void_p, _i64, _c_void_p]),
     "dora_fused_linear_fwd_workspace_size": (_size, [_i64, _i64]),
     "dora_fused_linear_fwd": (
         ctypes.c_int,
@@ -186,6 +191,24 @@ def dora_status_string(status: int) -> str:
 
 def dora_factored_norm(W, A, B, s: float, n_out=None, workspace=None, stream=None):
     """n = ||W + s B A||_row as fp32 [d_out] (factored; no dense B A)."""
+    return _factored_norm(W, A, B, s, n_out, workspace, stream, squared=False)
+
+
+def dora_factored_norm_sq(W, A, B, s: float, n2_out=None, workspace=None, stream=None):
+    """n^2 = ||W + s B A||_row^2 as summed (no sqrt, no clamp): a d_in shard's share."""
+    return _factored_norm(W, A, B, s, n2_out, workspace, stream, squared=True)
+
+
+def dora_norm_finish(n, stream=None):
+    """n = sqrt(max(n, 0)) in place (after summing dora_factored_norm_sq shares)."""
+    _dense_cuda(n)
+    if n.dtype != torch.float32 or n.dim() != 1:
+        raise TypeError("n must be a 1-D fp32 tensor")
+    _check(lib().dora_norm_finish(_ptr(n), n.numel(), _stream(stream)), "dora_norm_finish")
+    return n
+
+
+def _factored_norm(W, A, B, s, n_out, workspace, stream, squared):
     _dense_cuda(W, A, B, n_out, workspace)
     d_out, d_in = W.shape
     r = A.shape[0]
@@ -198,11 +221,12 @@ def dora_factored_norm(W, A, B, s: float, n_out=None, workspace=None, stream=Non
     need = dora_factored_norm_workspace_size(d_out, d_in, r, W.dtype)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
-    st = lib().dora_factored_norm(
+    fn = lib().dora_factored_norm_sq if squared else lib().dora_factored_norm
+    st = fn(
         _ptr(W), _ptr(A), _ptr(B), d_out, d_in, r, float(s), _dt(W), _ptr(n_out),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream),
     )
-    _check(st, "dora_factored_norm")
+    _check(st, "dora_factored_norm_sq" if squared else "dora_factored_norm")
     return n_out
 
 

@@ -89,6 +89,22 @@ typedef struct {
   float* n_out;
 } dora_norm_problem;
 
+/* dora_factored_norm without the final square root: n2_out[i] is
+ * ||W_i||^2 + 2s <B_i, U_i> + s^2 B_i G B_i^T as summed, not clamped.  Every
+ * term is a sum over d_in, so when W and A are split along d_in across ranks
+ * (a row-parallel layer), each rank's n2 over its own columns is its share of
+ * the full n^2: summing the shares (one all-reduce of d_out fp32) and applying
+ * dora_norm_finish gives the norm of the whole layer.  Arguments, workspace
+ * and errors as dora_factored_norm. */
+DORA_API int dora_factored_norm_sq(const void* W, const void* A, const void* B, int64_t d_out, int64_t d_in,
+                                   int64_t r, float s, dora_dtype dt, float* n2_out, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
+/* n[i] = sqrt(max(n[i], 0)) in place for i < d_out (fp32, 4-byte aligned):
+ * the last step after summing dora_factored_norm_sq shares.  d_out == 0 does
+ * nothing.  Asynchronous on `stream`. */
+DORA_API int dora_norm_finish(float* n, int64_t d_out, void* stream);
+
 /* Bytes of workspace dora_factored_norm_batched needs for these modules
  * (`problems`: host array of `count`); 0 for invalid arguments. */
 DORA_API size_t dora_factored_norm_batched_workspace_size(const dora_norm_problem* problems, int count, dora_dtype dt);

@@ -280,3 +280,16 @@ def test_norm_bwd_workspace_has_no_dense_term(lib):
         ws = lib.dora_factored_norm_bwd_workspace_size(d_out, d_in, r)
         assert ws < d_out * d_in * 2 // 4  # O(r d_out + r^2): 22.6 MB vs the dense 134 MB at 8192^2, r = 384
         assert lib.dora_factored_norm_bwd_workspace_size(d_out, 2 * d_in, r) == ws  # independent of d_in
+
+
+def test_norm_sq_and_finish_argument_errors(lib):
+    f = lib.dora_factored_norm_sq
+    assert f(FAKE, FAKE, FAKE, 64, 128, 16, 0.5, D.DORA_BF16, None, FAKE, 1 << 30, None) == D.DORA_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 64, 128, 12, 0.5, D.DORA_BF16, FAKE, FAKE, 1 << 30, None) == D.DORA_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, 64, 128, 16, 0.5, D.DORA_BF16, FAKE, FAKE, 0, None) == D.DORA_ERR_WORKSPACE
+    assert f(FAKE, FAKE, FAKE, 0, 128, 16, 0.5, D.DORA_BF16, FAKE, FAKE, 0, None) == D.DORA_OK
+    g = lib.dora_norm_finish
+    assert g(None, 8, None) == D.DORA_ERR_INVALID_ARG
+    assert g(FAKE, -1, None) == D.DORA_ERR_INVALID_ARG
+    assert g(ctypes.c_void_p(0x10002), 8, None) == D.DORA_ERR_UNSUPPORTED
+    assert g(None, 0, None) == D.DORA_OK
