@@ -145,3 +145,18 @@ def test_fused_linear_no_output_channels():
     x, W, A, B, b, m, n, s = _case(64, 128, 256, 16)
     y = D.dora_fused_linear_fwd(x, W[:0].contiguous(), A, B[:0].contiguous(), m[:0], n[:0], s)
     assert y.shape == (64, 0)
+
+
+def test_fused_linear_allocates_nothing():
+    # with the caller's workspace and output, the call allocates no device memory
+    x, W, A, B, b, m, n, s = _case(512, 2048, 1024, 384)
+    y = torch.empty(512, 1024, dtype=torch.bfloat16, device=DEV)
+    ws = torch.empty(D.dora_fused_linear_fwd_workspace_size(512, 384), dtype=torch.uint8, device=DEV)
+    D.dora_fused_linear_fwd(x, W, A, B, m, n, s, bias=b, y=y, workspace=ws)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        D.dora_fused_linear_fwd(x, W, A, B, m, n, s, bias=b, y=y, workspace=ws)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0

@@ -148,3 +148,18 @@ def test_norm_bwd_large_rank(r):
     rA, rB = oracle.norm_backward(P.f64(W), P.f64(A), P.f64(B), 0.5, P.f64(n), P.f64(d_n))
     assert_grad_close(dA, rA, "dA")
     assert_grad_close(dB, rB, "dB")
+
+
+def test_norm_bwd_allocates_nothing_and_has_no_dense_term():
+    # the dense B A of this shape would be 8 MB of bf16; the call allocates nothing
+    W, A, B, n, d_n = _case(2048, 2048, 384, 0.5)
+    dA = torch.empty(384, 2048, device=DEV)
+    dB = torch.empty(2048, 384, device=DEV)
+    ws = torch.empty(D.dora_factored_norm_bwd_workspace_size(2048, 2048, 384), dtype=torch.uint8, device=DEV)
+    D.dora_factored_norm_bwd(W, A, B, 0.5, n, d_n, dA=dA, dB=dB, workspace=ws)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        D.dora_factored_norm_bwd(W, A, B, 0.5, n, d_n, dA=dA, dB=dB, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
