@@ -229,6 +229,7 @@ def run_ours(args, rank, world, local_rank):
     # ---- end to end through the Python API with pinned host buffers
     e2e = run_e2e(args, D, dev, wl, W, A, B, m, base, lora, dy, n, y, d_base, d_lora, d_m, ws_n, ws_b, world)
     ctx = rank == 0 and not getattr(args, "no_context", False)
+    bf16_ctx = ctx and wl.dtype == "bf16"  # the fused linear and the norm backward take bf16 only
     # each context measurement starts from an idle GPU (a short host pause),
     # and the power-hungry fused-linear GEMMs run last
     def idle_then(f):
@@ -238,8 +239,8 @@ def run_ours(args, rank, world, local_rank):
 
     dense = idle_then(lambda: run_dense_comparator(D, dev, W, A, B, s, ws_n)) if ctx else None
     batched = idle_then(lambda: run_batched_context(D, dev)) if ctx else None
-    norm_bwd = idle_then(lambda: run_norm_backward_context(D, dev, wl, W, A, B, n)) if ctx else None
-    fused = idle_then(lambda: run_fused_linear_context(D, dev, wl, W, A, B, m, n)) if ctx else None
+    norm_bwd = idle_then(lambda: run_norm_backward_context(D, dev, wl, W, A, B, n)) if bf16_ctx else None
+    fused = idle_then(lambda: run_fused_linear_context(D, dev, wl, W, A, B, m, n)) if bf16_ctx else None
     return dict(t_total=t_total, t_norm=t_norm, t_fwd=t_fwd, t_bwd=t_bwd, clocks=clocks, status=status, e2e=e2e,
                 wl=wl, dense=dense, batched=batched, fused=fused, norm_bwd=norm_bwd)
 
