@@ -7,6 +7,12 @@
  * is computed from base, cross and Gram terms without forming B A, and the
  * magnitude rescaling is composed with the base and LoRA outputs in one pass.
  *
+ * Entry points: the factored norm (one module, many modules at once, or a
+ * d_in shard's squared share), the compose forward and its backward with the
+ * norm detached (with or without a base-layer bias, with or without a
+ * workspace), the compose fused into the GEMMs that produce its inputs, and
+ * the norm's own gradients into A and B for training with the norm attached.
+ *
  * Conventions shared by every call
  * --------------------------------
  *  - Layout: dense, row-major, contiguous.  W is [d_out, d_in] (frozen base
@@ -18,9 +24,10 @@
  *  - Pointers are device pointers unless stated.  The caller owns and allocates
  *    every buffer, including the workspace; the library never allocates device
  *    memory, so no O(d_out * d_in) temporary ever exists.
- *  - bf16 requires 16-byte aligned pointers, d_in and d_out multiples of 8 and
- *    r a multiple of 16 (else DORA_ERR_UNSUPPORTED).  fp32 accepts any shape
- *    with 4-byte aligned pointers.
+ *  - bf16 requires 16-byte aligned pointers and d_in, d_out multiples of 8;
+ *    the factored norm also needs r a multiple of 16, the other calls state
+ *    their own rules (else DORA_ERR_UNSUPPORTED).  fp32 accepts any shape with
+ *    4-byte aligned pointers where a call takes fp32.
  *  - stream is a cudaStream_t passed as void* (NULL = legacy default stream).
  *    Every call is asynchronous on it and returns once the work is enqueued.
  *  - Errors: argument errors are detected on the host before anything is
@@ -51,7 +58,7 @@ typedef enum { DORA_BF16 = 0, DORA_F32 = 1 } dora_dtype;
 
 typedef enum {
   DORA_OK = 0,
-  DORA_ERR_INVALID_ARG = 1, /* null pointer, negative size, r > d_in ... */
+  DORA_ERR_INVALID_ARG = 1, /* null pointer, negative size ... */
   DORA_ERR_UNSUPPORTED = 2, /* alignment / shape / dtype this build does not handle */
   DORA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than the size query */
   DORA_ERR_CUDA = 4,        /* a CUDA runtime call failed (launch, attribute ...) */
@@ -77,18 +84,6 @@ DORA_API int dora_factored_norm(const void* W, const void* A, const void* B, int
                        float s, dora_dtype dt, float* n_out, void* workspace, size_t workspace_bytes,
                        void* stream);
 
-/* One adapted module for dora_factored_norm_batched: the arguments of
- * dora_factored_norm for that module (device pointers, row-major layouts as
- * above; n_out is overwritten). */
-typedef struct {
-  const void* W;
-  const void* A;
-  const void* B;
-  int64_t d_out, d_in, r;
-  float s;
-  float* n_out;
-} dora_norm_problem;
-
 /* dora_factored_norm without the final square root: n2_out[i] is
  * ||W_i||^2 + 2s <B_i, U_i> + s^2 B_i G B_i^T as summed, not clamped.  Every
  * term is a sum over d_in, so when W and A are split along d_in across ranks
@@ -104,6 +99,18 @@ DORA_API int dora_factored_norm_sq(const void* W, const void* A, const void* B, 
  * the last step after summing dora_factored_norm_sq shares.  d_out == 0 does
  * nothing.  Asynchronous on `stream`. */
 DORA_API int dora_norm_finish(float* n, int64_t d_out, void* stream);
+
+/* One adapted module for dora_factored_norm_batched: the arguments of
+ * dora_factored_norm for that module (device pointers, row-major layouts as
+ * above; n_out is overwritten). */
+typedef struct {
+  const void* W;
+  const void* A;
+  const void* B;
+  int64_t d_out, d_in, r;
+  float s;
+  float* n_out;
+} dora_norm_problem;
 
 /* Bytes of workspace dora_factored_norm_batched needs for these modules
  * (`problems`: host array of `count`); 0 for invalid arguments. */
