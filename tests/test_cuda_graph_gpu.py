@@ -1,8 +1,8 @@
 """The library's calls captured into CUDA graphs and replayed.
 
 Every entry point takes its stream and all of its buffers from the caller and
-launches a fixed sequence (programmatic dependent launches, clusters, a
-memset node), so a step can be captured once and replayed with new input
+launches a fixed sequence (programmatic dependent launches, clusters, no
+memset nodes), so a step can be captured once and replayed with new input
 values written into the same buffers.  Each replay must reproduce, bit for
 bit, what eager calls on the same inputs give (every path sums in a fixed
 order).
