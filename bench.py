@@ -14,7 +14,10 @@ roofline fraction ride along in the same JSON line.  Multi-GPU runs are
 independent replicas (weak scaling): the path has no exchange step.
 
 ``--impl reference`` times the fp64 CPU oracle (the reference arm) on the
-host cores on a bounded sample of the same workload.
+host cores on a bounded sample of the same workload.  ``--sweep`` runs the
+rank/shape sweep instead (the norm over ranks 16..768, the compose over
+token counts 1024..65536, each call timed alone after an L2 flush) and
+prints its points.
 """
 
 from __future__ import annotations
@@ -653,6 +656,102 @@ def build_line(args, res, N, peaks, peak_src, traffic, cpu):
     return line
 
 
+# ------------------------------------------------------------------ sweep
+SWEEP_FLUSH_BYTES = 256 << 20  # twice the 126 MB L2
+
+
+class L2Flush:
+    """Writes one buffer larger than L2, then reads another: the read evicts
+    the written lines (their write-back happens here, untimed) and leaves L2
+    holding clean lines of the second buffer, so the next call neither finds
+    its inputs in L2 nor pays for someone else's dirty lines."""
+
+    def __init__(self, dev):
+        self.w = torch.empty(SWEEP_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        self.r = torch.zeros(SWEEP_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        self.acc = torch.empty((), dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        self.w.fill_(1.0)
+        torch.sum(self.r, dim=0, out=self.acc)
+
+
+def time_alone(f, reps, flush, stream):
+    """Median CUDA-event time (s) of f() over reps calls, each timed alone on
+    ``stream`` after ``flush()``, which is not timed."""
+    for _ in range(3):
+        flush()
+        f()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for e0, e1 in evs:
+        flush()
+        e0.record(stream)
+        f()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return statistics.median(e0.elapsed_time(e1) for e0, e1 in evs) * 1e-3
+
+
+def run_sweep(args):
+    """The rank/shape sweep workload on one GPU: the factored norm at
+    d_out = d_in = 8192 for every rank of RANK_SWEEP, then the compose forward
+    and backward at d_out = 8192 for every token count of TOKEN_SWEEP (m, n
+    with m / n = 1 + N(0, 1e-4)).  Each point's time is the median of calls
+    timed alone after an L2 flush (L2Flush); each point gives its throughput and its
+    fraction of the roofline time (the slower of its algorithmic FLOPs at the
+    measured bf16 peak and its algorithmic bytes at the measured copy
+    bandwidth).  Prints one JSON line {"sweep": [...], ...}; it is not the
+    benchmark line."""
+    from factored_weight_norm_b200 import dora as D
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    peaks, peak_src = load_peaks()
+    reps = max(5, min(args.steps, 50))
+    flush = L2Flush(dev)
+    pts = []
+    sampler = ClockSampler(0)
+    sampler.start()
+    for wl in WL.RANK_SWEEP:
+        W, A, B, _ = WL.make_weights(wl, dev)
+        n = torch.empty(wl.d_out, dtype=torch.float32, device=dev)
+        ws = torch.empty(D.dora_factored_norm_workspace_size(wl.d_out, wl.d_in, wl.r), dtype=torch.uint8,
+                         device=dev)
+        t = time_alone(lambda: D.dora_factored_norm(W, A, B, wl.s, n_out=n, workspace=ws), reps, flush, stream)
+        fl, by = norm_flops(wl.d_out, wl.d_in, wl.r), norm_bytes(wl.d_out, wl.d_in, wl.r)
+        t_roof = max(fl / (peaks["bf16_tflops"] * 1e12), by / (peaks["hbm_gbs"] * 1e9))
+        pts.append({"op": "factored_norm", "d_out": wl.d_out, "d_in": wl.d_in, "r": wl.r, "us": t * 1e6,
+                    "tflops": fl / t * 1e-12, "gbs": by / t * 1e-9,
+                    "bound": "tensor" if fl / (peaks["bf16_tflops"] * 1e12) >= by / (peaks["hbm_gbs"] * 1e9)
+                    else "hbm", "roofline_frac": t_roof / t})
+        del W, A, B, ws
+    base_wl = WL.TOKEN_SWEEP[0]
+    W, A, B, _ = WL.make_weights(base_wl, dev)
+    m, n = WL.make_near_unity_mn(base_wl, W, dev)
+    for wl in WL.TOKEN_SWEEP:
+        _, base, lora = WL.make_activations(wl, W, A, B, dev)
+        dy = WL.make_grad(wl, dev)
+        y, d_base, d_lora = torch.empty_like(base), torch.empty_like(base), torch.empty_like(base)
+        d_m = torch.empty(wl.d_out, dtype=torch.float32, device=dev)
+        ws = torch.empty(D.dora_compose_bwd_workspace_size(wl.tokens, wl.d_out), dtype=torch.uint8, device=dev)
+        t_f = time_alone(lambda: D.dora_compose_fwd(base, lora, m, n, wl.s, y=y), reps, flush, stream)
+        t_b = time_alone(lambda: D.dora_compose_bwd(dy, base, lora, m, n, wl.s, d_base, d_lora, d_m, ws), reps,
+                         flush, stream)
+        for op, t, by in (("compose_fwd", t_f, fwd_bytes(wl.tokens, wl.d_out)),
+                          ("compose_bwd", t_b, bwd_bytes(wl.tokens, wl.d_out))):
+            pts.append({"op": op, "tokens": wl.tokens, "d_out": wl.d_out, "us": t * 1e6, "gbs": by / t * 1e-9,
+                        "bound": "hbm", "roofline_frac": by / t * 1e-9 / peaks["hbm_gbs"]})
+        del base, lora, dy, y, d_base, d_lora, ws
+    clocks = sampler.stop()
+    status = D.dora_device_status()
+    print(json.dumps({"sweep": pts, "reps_per_point": reps, "l2": "before every timed call 256 MB written, then another 256 MB read",
+                      "peaks": {"bf16_tflops": peaks["bf16_tflops"], "hbm_gbs": peaks["hbm_gbs"],
+                                "source": peak_src}, "clocks": clocks, "device_status": status}), flush=True)
+    return 0 if status == D.DORA_OK else 1
+
+
 # ------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -667,8 +766,13 @@ def main():
     ap.add_argument("--no-context", action="store_true",
                     help="skip the context measurements after the timed step (dense comparator, many modules, "
                          "fused linear, attached-norm backward), e.g. for a profiler's launch list")
+    ap.add_argument("--sweep", action="store_true",
+                    help="run the rank/shape sweep (norm over ranks, compose over token counts) on one GPU "
+                         "and print its points instead of the benchmark line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.sweep:
+        return run_sweep(args)
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

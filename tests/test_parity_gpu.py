@@ -35,6 +35,7 @@ SMALL_NORM = [
     (128, 64, 16),      # one tile, one K block, smallest rank
     (256, 512, 64),
     (300, 520, 48),     # ragged M tile and ragged K block
+    (136, 200, 112),    # rank below one box: N-side boxes of r rows, ragged M tile
     (1000, 1000, 128),
     (512, 1024, 384),   # headline rank, two MMA pieces (256 + 128)
     (384, 640, 256),
