@@ -771,14 +771,16 @@ def main():
                          "and print its points instead of the benchmark line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
-    if args.sweep:
-        return run_sweep(args)
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.sweep:
+        if world > 1:
+            raise SystemExit("--sweep measures one GPU; run it without torchrun")
+        return run_sweep(args)
 
     if world > 1:
         import datetime

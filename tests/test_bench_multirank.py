@@ -106,3 +106,16 @@ def test_reference_arm_runs_on_rank_zero_only(two_ranks):
     assert two_ranks[1]["ref_rc"] == 0
     assert two_ranks[1]["ref_out"] == ""
     assert "line" not in two_ranks[1]
+
+
+def test_sweep_refuses_several_ranks():
+    """The sweep times one GPU; under torchrun every rank would otherwise pick
+    cuda:0, so a world size above one is refused before any device work."""
+    import subprocess
+    import sys
+
+    env = dict(os.environ, RANK="0", WORLD_SIZE="2", LOCAL_RANK="0")
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--sweep"], env=env, capture_output=True,
+                       text=True, timeout=300)
+    assert p.returncode != 0
+    assert "one GPU" in p.stderr
