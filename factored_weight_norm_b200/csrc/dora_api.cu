@@ -309,8 +309,8 @@ int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_
   na.kb_total = p.kb_total;
   na.units = p.units;
   na.stage_bytes = static_cast<uint32_t>(kBoxBytes * (1 + cdiv(p.chunk_n, kBoxRows)));
-  const size_t fixed = 1024 + 64 + 16;
-  na.stages = static_cast<int>(std::min<size_t>(kMaxStages, (dev->smem_optin - fixed) / (na.stage_bytes + 16)));
+  na.stages = static_cast<int>(
+      std::min<size_t>(kMaxStages, (dev->smem_optin - kNormTcSmemFixed) / (na.stage_bytes + 16)));
   if (na.stages < 2) return DORA_ERR_UNSUPPORTED;
   uint32_t cols = 32;
   while (cols < static_cast<uint32_t>(p.chunk_n)) cols <<= 1;
@@ -324,8 +324,8 @@ int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_
   na.squared = squared ? 1 : 0;
   const int grid = static_cast<int>(std::min<long long>({static_cast<long long>(dev->num_sms), p.units, kMaxGrid}));
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kNormThreads);
-  cfg.dynamicSmemBytes = static_cast<size_t>(na.stages) * na.stage_bytes + (2 * na.stages + 3) * 8 + 16 + 1024;
+  cfg.blockDim = dim3(kNormTcThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(na.stages) * (na.stage_bytes + 16) + kNormTcSmemFixed;
   if (cudaLaunchKernelEx(&cfg, norm_tc_kernel, tmW, tmA, tmB, tmG, na) != cudaSuccess) return DORA_ERR_CUDA;
   return launch_error();
 }

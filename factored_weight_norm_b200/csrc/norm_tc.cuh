@@ -20,9 +20,10 @@
 //                      block) units; each CTA owns a contiguous unit range and
 //                      starts streaming W before the Gram kernels finish (it
 //                      only waits for them before its first K-extension block).
-//                      Epilogue: ||W_i||^2 from the shared-memory W stages;
-//                      B's rows arrive through the same TMA ring after each
-//                      segment and are dotted with V_i read from TMEM; one
+//                      Two warps sum ||W_i||^2 from the shared-memory W
+//                      stages; at each segment end B's rows arrive through
+//                      the same TMA ring and four epilogue warps dot them
+//                      with V_i read from TMEM; one
 //                      fp32 partial per (row, segment); the last warp to finish
 //                      an M tile sums its partials in fixed order and writes
 //                      n = sqrt(max(., 0)).
@@ -36,7 +37,18 @@ constexpr int kBM = 128;              // rows per M tile (TMEM lanes)
 constexpr int kBK = 64;               // bf16 along K per 128-byte swizzled row
 constexpr int kBoxRows = 128;         // rows per TMA box
 constexpr int kBoxBytes = kBoxRows * 128;
-constexpr int kNormThreads = 192;     // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kNormThreads = 192;     // Gram kernels: warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+// norm_tc_kernel: warp 0 TMA, warp 1 MMA, warps 2..5 TMEM epilogue at segment
+// ends, warps 6 and 7 ||W_i||^2 over every W stage.  A warp runs on the SM
+// sub-partition (warp index mod 4) whose TMEM lane quarter it may read, so one
+// epilogue warp always shares the MMA thread's sub-partition; the per-stage
+// work goes to warps 6 and 7 (sub-partitions 2 and 3) so that it does not
+// compete with the MMA thread for issue slots.
+constexpr int kNormTcThreads = 256;
+// shared memory besides the stages: 1024-byte alignment slack, five single
+// mbarriers, the TMEM address and abort flag (16 bytes), the W^2 hand-off
+// (kBM floats); each stage adds its two mbarriers
+constexpr int kNormTcSmemFixed = 1024 + 5 * 8 + 16 + kBM * 4;
 constexpr int kMaxChunkN = 512;       // TMEM columns
 constexpr int kMaxStages = 8;
 constexpr int kStatusTimeout = 5;     // == DORA_ERR_TIMEOUT
@@ -144,7 +156,7 @@ __device__ __forceinline__ int b_stages(const NormArgs& a, int n_this) {
 }
 
 // ===================================================================== norm
-__global__ void __launch_bounds__(kNormThreads, 1)
+__global__ void __launch_bounds__(kNormTcThreads, 1)
     norm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA,
                    const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmG,
                    const NormArgs a) {
@@ -157,8 +169,11 @@ __global__ void __launch_bounds__(kNormThreads, 1)
   uint64_t* tmem_full = empty + a.stages;
   uint64_t* tmem_empty = tmem_full + 1;
   uint64_t* drain = tmem_empty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* w2_full = drain + 1;   // the W^2 warps' row sums of a segment are in w2
+  uint64_t* w2_empty = w2_full + 1;  // the epilogue warps have read them
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(w2_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* w2 = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(w2_empty + 1) + 16);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -172,11 +187,18 @@ __global__ void __launch_bounds__(kNormThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.stages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + 4);  // MMA warp + one arrive per epilogue warp
+      // W stages: the MMA commit + 3 from each W^2 warp; segment-end B
+      // stages: the MMA warp + one arrive per epilogue and per W^2 warp.
+      // Every warp that waits on a stage's fills also arrives on its
+      // releases, so no fill can complete twice before a waiter sees it
+      // (a parity wait cannot tell phase k from phase k + 2).
+      mbar_init(&empty[s], 1 + 4 + 2);
     }
     mbar_init(tmem_full, 1);
     mbar_init(tmem_empty, 4);
     mbar_init(drain, 1);
+    mbar_init(w2_full, 2);
+    mbar_init(w2_empty, 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -341,19 +363,20 @@ __global__ void __launch_bounds__(kNormThreads, 1)
       mma_commit(drain);
       mbar_wait(drain, 0, limit);
     }
-  } else {
-    // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
-    const int row_local = q * 32 + lane;
-    const uint32_t tmem_lane = tmem + (static_cast<uint32_t>(q * 32) << 16);
+  } else if (warp >= 6) {
+    // ------------------------------------------------------- ||W_i||^2 warps
+    // Warp 6 sums rows 0..63 of every W stage, warp 7 rows 64..127 (lane l:
+    // rows l and l + 32 of its half), and releases the stage with a triple
+    // arrival; at each segment end the row sums go to the epilogue warps
+    // through shared memory.  The sum ignores the chunk order, and visiting
+    // chunk (j ^ row % 8) keeps the eight rows of a quarter-warp on distinct
+    // banks.
+    const int r0 = (warp - 6) * 64 + lane;
     int stage = 0;
     uint32_t phase = 0;
     int seg = 0;
-    float base_acc = 0.f;
-    bool deps_ready = false;
-    auto release = [&]() {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[stage]);
+    float acc0 = 0.f, acc1 = 0.f;
+    auto step = [&]() {
       if (++stage == a.stages) {
         stage = 0;
         phase ^= 1u;
@@ -366,15 +389,67 @@ __global__ void __launch_bounds__(kNormThreads, 1)
         break;
       }
       if (x.ch == 0 && x.kb < a.kb_main) {
-        // ||W_i||^2 from the swizzled W stage; the sum ignores the chunk
-        // order, and visiting chunk (j ^ row % 8) keeps the eight rows of a
-        // quarter-warp on distinct banks.
         const uint8_t* tile = smem + stage * a.stage_bytes;
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          base_acc += sumsq_bf16x8(*reinterpret_cast<const uint4*>(tile + sw128_chunk(row_local, j)));
+        for (int j = 0; j < 8; ++j) {
+          acc0 += sumsq_bf16x8(*reinterpret_cast<const uint4*>(tile + sw128_chunk(r0, j)));
+          acc1 += sumsq_bf16x8(*reinterpret_cast<const uint4*>(tile + sw128_chunk(r0 + 32, j)));
+        }
       }
-      release();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cnt(&empty[stage], 3);
+      step();
+      if (!x.seg_last(a)) continue;
+      // the segment-end B stages: the epilogue warps read them; these warps
+      // only keep their place in the ring
+      const int nbst = b_stages(a, x.n_this);
+      bool ok = true;
+      for (int i = 0; i < nbst; ++i) {
+        if (__any_sync(0xffffffffu, !mbar_wait(&full[stage], phase, limit))) {
+          if (lane == 0) record_timeout(a.status, abort_flag);
+          ok = false;
+          break;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[stage]);
+        step();
+      }
+      if (!ok) break;
+      if (seg > 0 && !mbar_wait_warp(w2_empty, static_cast<uint32_t>((seg - 1) & 1), limit)) {
+        if (lane == 0) record_timeout(a.status, abort_flag);
+        break;
+      }
+      w2[r0] = acc0;
+      w2[r0 + 32] = acc1;
+      acc0 = acc1 = 0.f;
+      __threadfence_block();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(w2_full);
+      ++seg;
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row_local = q * 32 + lane;
+    const uint32_t tmem_lane = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    int stage = 0;
+    uint32_t phase = 0;
+    int seg = 0;
+    bool deps_ready = false;
+    auto step = [&]() {
+      if (++stage == a.stages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    };
+    auto release = [&]() {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);
+      step();
+    };
+    UnitIter x;
+    for (x.start(a, u_begin, u_end); x.valid(); x.next(a)) {
+      step();  // the W stages are the MMA thread's and the W^2 warps'
       if (!x.seg_last(a)) continue;
 
       // ---- segment epilogue: <B_i, V_i> over this chunk's columns
@@ -417,8 +492,15 @@ __global__ void __launch_bounds__(kNormThreads, 1)
       if (lane == 0) mbar_arrive(tmem_empty);
       ++seg;
 
+      // this segment's ||W_i||^2 from the W^2 warps
+      if (!mbar_wait_warp(w2_full, static_cast<uint32_t>((seg - 1) & 1), limit)) {
+        if (lane == 0) record_timeout(a.status, abort_flag);
+        break;
+      }
+      const float base_acc = w2[row_local];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(w2_empty);
       const float partial = base_acc + a.two_s * dot;
-      base_acc = 0.f;
       if (!deps_ready) {
         grid_dep_wait();  // counters are zeroed by the Gram reduction kernel
         deps_ready = true;
