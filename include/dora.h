@@ -35,6 +35,11 @@
  *    DORA_ERR_WORKSPACE.  A failed launch returns DORA_ERR_CUDA.  Kernels that
  *    wait on other threads bound every wait; if one gives up it records
  *    DORA_ERR_TIMEOUT in a device-side word that dora_device_status() reports.
+ *    The outputs of that call are undefined.  Nothing in a workspace has to be
+ *    cleared by the caller: the compose backward's arrival counters carry a
+ *    tag that is new for every call.  A CUDA graph replays its captured tag,
+ *    so after a replay of a compose backward that timed out, re-capture the
+ *    graph (or zero that workspace) before replaying it.
  *  - Outputs are overwritten, never accumulated into.  Results are
  *    deterministic: every reduction runs in a fixed order.
  */
