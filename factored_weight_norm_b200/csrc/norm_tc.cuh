@@ -23,10 +23,9 @@
 //                      Two warps sum ||W_i||^2 from the shared-memory W
 //                      stages; at each segment end B's rows arrive through
 //                      the same TMA ring and four epilogue warps dot them
-//                      with V_i read from TMEM; one
-//                      fp32 partial per (row, segment); the last warp to finish
-//                      an M tile sums its partials in fixed order and writes
-//                      n = sqrt(max(., 0)).
+//                      with V_i read from TMEM; one fp32 partial per (row,
+//                      segment); the last warp to finish an M tile sums its
+//                      partials in fixed order and writes n = sqrt(max(., 0)).
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -37,7 +36,7 @@ constexpr int kBM = 128;              // rows per M tile (TMEM lanes)
 constexpr int kBK = 64;               // bf16 along K per 128-byte swizzled row
 constexpr int kBoxRows = 128;         // rows per TMA box
 constexpr int kBoxBytes = kBoxRows * 128;
-constexpr int kNormThreads = 192;     // Gram kernels: warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kNormThreads = 192;     // Gram and batched kernels: warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 // norm_tc_kernel: warp 0 TMA, warp 1 MMA, warps 2..5 TMEM epilogue at segment
 // ends, warps 6 and 7 ||W_i||^2 over every W stage.  A warp runs on the SM
 // sub-partition (warp index mod 4) whose TMEM lane quarter it may read, so one
