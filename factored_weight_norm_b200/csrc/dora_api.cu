@@ -230,14 +230,19 @@ int ctas_per_sm(K kernel, int threads) {
   return n;
 }
 
-// Row chunks of the compose backward for `strips` column strips: as many as
-// one wave of `slots` resident CTAs holds, at most k_max, at least one.  One
-// wave of longer CTAs measured faster than two waves of shorter ones (each
-// CTA pays a ramp-up of its loads and a partial-sum write at its end): at
-// d_out = 8192, 110.6 against 112.6 us for 8192 tokens, 57.3 against 59.4 us
-// for 4096.
-long long bwd_chunks(long long strips, long long slots, long long k_max) {
-  return std::max<long long>(1, std::min<long long>(slots / strips, k_max));
+// Row chunks of the compose backward for `strips` column strips (at most
+// k_max, at least one): as many as one wave of `slots` resident CTAs holds
+// while that leaves each CTA at most kBwdWaveRows rows, else about two waves.
+// Measured at d_out = 8192: one wave of longer CTAs beats two waves of
+// shorter ones up to 8192 tokens (110.6 against 112.6 us; 57.3 against
+// 59.4 us at 4096), since each CTA pays a ramp-up of its loads and a
+// partial-sum write at its end; two waves win from 16384 tokens on (215.0
+// against 218.9 us; 848.8 against 869.4 us at 65536).
+constexpr long long kBwdWaveRows = 2048;
+long long bwd_chunks(long long strips, long long slots, long long tokens, long long k_max) {
+  long long k = std::max<long long>(1, slots / strips);
+  if (cdiv(tokens, k) > kBwdWaveRows) k = std::max<long long>(1, 2 * slots / strips);
+  return std::max<long long>(1, std::min<long long>(k, k_max));
 }
 
 int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_t d_in, int64_t r, float s,
@@ -663,7 +668,7 @@ int dora_compose_bwd_bias(const void* dy, const void* base_out, const void* lora
     occ = ctas_per_sm(compose_bwd_kernel<float, 4, false>, kBwdThreads);
   else
     occ = ctas_per_sm(compose_bwd_kernel<float, 1, false>, kBwdThreads);
-  const long long chunks = bwd_chunks(strips, static_cast<long long>(dev->num_sms) * occ,
+  const long long chunks = bwd_chunks(strips, static_cast<long long>(dev->num_sms) * occ, tokens,
                                       std::min<long long>(kMaxBwdChunks, cdiv(tokens, kBwdSlots)));
   const long long rows = cdiv(tokens, chunks);
   const long long chunks2 = cdiv(tokens, rows);
@@ -1139,7 +1144,7 @@ extern "C" int dora_compose_bwd_noalloc_bias(const void* dy, const void* base_ou
     occ = ctas_per_sm(compose_bwd_kernel<float, 4, false>, kBwdThreads);
   else
     occ = ctas_per_sm(compose_bwd_kernel<float, 1, false>, kBwdThreads);
-  const long long chunks = bwd_chunks(strips, static_cast<long long>(dev->num_sms) * occ,
+  const long long chunks = bwd_chunks(strips, static_cast<long long>(dev->num_sms) * occ, tokens,
                                       std::min<long long>(kNoallocChunks, cdiv(tokens, kBwdSlots)));
   const long long rows = cdiv(tokens, chunks);
   const long long chunks2 = cdiv(tokens, rows);
