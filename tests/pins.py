@@ -300,6 +300,8 @@ def pin_bias_layer(compose_forward, compose_backward, seed=6):
 def pin_norm_backward(norm_backward, seed=8):
     import torch
 
+    pin_hand_norm_backward(norm_backward)
+
     rng = np.random.default_rng(seed)
     for d_out, d_in, r in ((3, 4, 2), (5, 7, 3), (4, 9, 5)):
         W, A, B = tiny_case(rng, d_out, d_in, r)
@@ -344,6 +346,7 @@ def brute_layer(x, W, A, B, m, n, s, b):
 
 
 def pin_layer(linear_forward, compose_forward, seed=7):
+    pin_hand_layer(linear_forward)
     rng = np.random.default_rng(seed)
     for T, d_in, d_out, r in ((1, 1, 1, 1), (3, 5, 4, 2), (6, 9, 7, 3)):
         x = rng.standard_normal((T, d_in))
@@ -370,6 +373,27 @@ def pin_layer(linear_forward, compose_forward, seed=7):
 def load_hand_cases():
     with open(os.path.join(GOLDEN, "hand_cases.json")) as f:
         return json.load(f)["cases"]
+
+
+def pin_hand_layer(linear_forward):
+    """The adapted layer on the hand-worked case (exact in binary)."""
+    for case in load_hand_cases():
+        if "x" not in case:
+            continue
+        W, A, B, m, n, x, b = (np.array(case[k], dtype=np.float64) for k in ("W", "A", "B", "m", "n", "x", "bias"))
+        y = linear_forward(x, W, A, B, m, n, float(case["s"]), bias=b)
+        assert np.array_equal(np.asarray(y, float), np.array(case["y_layer"], dtype=np.float64)), case["name"]
+
+
+def pin_hand_norm_backward(norm_backward):
+    """Gradients of n w.r.t. A and B on the hand-worked case (exact in binary)."""
+    for case in load_hand_cases():
+        if "d_n" not in case:
+            continue
+        W, A, B, n, d_n = (np.array(case[k], dtype=np.float64) for k in ("W", "A", "B", "n", "d_n"))
+        dA, dB = norm_backward(W, A, B, float(case["s"]), n, d_n)
+        assert np.array_equal(np.asarray(dA, float), np.array(case["dA"], dtype=np.float64)), case["name"]
+        assert np.array_equal(np.asarray(dB, float), np.array(case["dB"], dtype=np.float64)), case["name"]
 
 
 def pin_hand_cases(row_norm, compose_forward, compose_backward):
