@@ -119,3 +119,17 @@ def test_sweep_refuses_several_ranks():
                        text=True, timeout=300)
     assert p.returncode != 0
     assert "one GPU" in p.stderr
+
+
+def test_line_has_every_contract_key(two_ranks):
+    line = two_ranks[0]["line"]
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+              "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks", "cpu_baseline"):
+        assert k in line, k
+    assert line["higher_is_better"] is True and line["steps"] == 7 and line["warmup"] == 3
+    assert "workload" in line["config"]
+    for k in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
+        assert k in line["roofline"], k
+    for k in ("value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"):
+        assert k in line["e2e"], k
+    assert line["gpu_launches"] > 0
