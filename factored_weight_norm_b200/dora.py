@@ -154,13 +154,51 @@ def _stream(stream=None):
 
 
 def _dense_cuda(*ts):
+    """Every tensor given is a contiguous CUDA tensor on the current device.
+
+    Kernels launch on the current device's stream and read their operands
+    there, so a tensor on another GPU (or the host) is refused before any
+    launch rather than read through a pointer that belongs elsewhere."""
+    cur = None
     for t in ts:
         if t is None:
             continue
         if not t.is_cuda:
             raise ValueError("tensors must live on a CUDA device")
+        if cur is None:
+            cur = torch.cuda.current_device()
+        if t.device.index != cur:
+            raise ValueError(f"tensor on {t.device} but the current device is cuda:{cur}")
         if not t.is_contiguous():
             raise ValueError("tensors must be contiguous (row-major)")
+
+
+def _like(ref, where: str, **named):
+    """Each named tensor (None skipped) has ref's shape and dtype."""
+    for name, t in named.items():
+        if t is None:
+            continue
+        if tuple(t.shape) != tuple(ref.shape):
+            raise ValueError(f"{where}: {name} has shape {tuple(t.shape)}, expected {tuple(ref.shape)}")
+        if t.dtype != ref.dtype:
+            raise TypeError(f"{where}: {name} is {t.dtype}, expected {ref.dtype}")
+
+
+def _vec_f32(d: int, where: str, **named):
+    """Each named tensor (None skipped) is fp32 of shape (d,)."""
+    for name, t in named.items():
+        if t is None:
+            continue
+        if tuple(t.shape) != (d,):
+            raise ValueError(f"{where}: {name} has shape {tuple(t.shape)}, expected ({d},)")
+        if t.dtype != torch.float32:
+            raise TypeError(f"{where}: {name} must be fp32, got {t.dtype}")
+
+
+def _acts2d(base_out, where: str):
+    if base_out.dim() != 2:
+        raise ValueError(f"{where}: activations must be 2-D [tokens, d_out], got {tuple(base_out.shape)}")
+    _dt(base_out)
 
 
 # ---------------------------------------------------------------- C names
@@ -201,21 +239,26 @@ def dora_factored_norm_sq(W, A, B, s: float, n2_out=None, workspace=None, stream
 
 def dora_norm_finish(n, stream=None):
     """n = sqrt(max(n, 0)) in place (after summing dora_factored_norm_sq shares)."""
-    _dense_cuda(n)
     if n.dtype != torch.float32 or n.dim() != 1:
         raise TypeError("n must be a 1-D fp32 tensor")
+    _dense_cuda(n)
     _check(lib().dora_norm_finish(_ptr(n), n.numel(), _stream(stream)), "dora_norm_finish")
     return n
 
 
 def _factored_norm(W, A, B, s, n_out, workspace, stream, squared):
-    _dense_cuda(W, A, B, n_out, workspace)
+    where = "dora_factored_norm_sq" if squared else "dora_factored_norm"
+    if W.dim() != 2 or A.dim() != 2 or B.dim() != 2:
+        raise ValueError(f"{where}: W, A and B must be 2-D")
     d_out, d_in = W.shape
     r = A.shape[0]
     if A.shape != (r, d_in) or B.shape != (d_out, r):
         raise ValueError(f"shape mismatch: W {tuple(W.shape)}, A {tuple(A.shape)}, B {tuple(B.shape)}")
     if not (W.dtype == A.dtype == B.dtype):
         raise TypeError("W, A and B must share one dtype")
+    _dt(W)
+    _vec_f32(d_out, where, n_out=n_out)
+    _dense_cuda(W, A, B, n_out, workspace)
     if n_out is None:
         n_out = torch.empty(d_out, dtype=torch.float32, device=W.device)
     need = dora_factored_norm_workspace_size(d_out, d_in, r, W.dtype)
@@ -232,14 +275,15 @@ def _factored_norm(W, A, B, s, n_out, workspace, stream, squared):
 
 def _problem_array(modules, n_outs):
     arr = (NormProblem * len(modules))()
+    dt0 = modules[0][0].dtype if modules else None
     for i, ((W, A, B, s), n) in enumerate(zip(modules, n_outs)):
-        _dense_cuda(W, A, B, n)
         d_out, d_in = W.shape
         r = A.shape[0]
         if A.shape != (r, d_in) or B.shape != (d_out, r) or n.shape != (d_out,):
             raise ValueError(f"module {i}: shape mismatch: W {tuple(W.shape)}, A {tuple(A.shape)}, B {tuple(B.shape)}")
-        if not (W.dtype == A.dtype == B.dtype) or n.dtype != torch.float32:
-            raise TypeError(f"module {i}: W, A, B share one dtype; n is fp32")
+        if not (W.dtype == A.dtype == B.dtype == dt0) or n.dtype != torch.float32:
+            raise TypeError(f"module {i}: W, A, B share the first module's dtype; n is fp32")
+        _dense_cuda(W, A, B, n)
         arr[i] = NormProblem(W.data_ptr(), A.data_ptr(), B.data_ptr(), d_out, d_in, r, float(s), n.data_ptr())
     return arr
 
@@ -275,7 +319,6 @@ def dora_factored_norm_batched(modules, n_outs=None, workspace=None, stream=None
 def _check_bias(bias, base_out, name):
     if bias is None:
         return
-    _dense_cuda(bias)
     if bias.shape != (base_out.shape[1],):
         raise ValueError(f"bias must have shape (d_out,) in {name}")
     if bias.dtype != base_out.dtype:
@@ -287,13 +330,13 @@ def dora_compose_fwd(base_out, lora_out, m, n, s: float, y=None, stream=None, bi
 
     base_out is the base layer's output including its bias b (``bias``,
     ``None`` for a layer without one)."""
-    _dense_cuda(base_out, lora_out, m, n, y)
+    where = "dora_compose_fwd"
+    _acts2d(base_out, where)
     tokens, d_out = base_out.shape
-    if lora_out.shape != base_out.shape or m.shape != (d_out,) or n.shape != (d_out,):
-        raise ValueError("shape mismatch in dora_compose_fwd")
-    if m.dtype != torch.float32 or n.dtype != torch.float32:
-        raise TypeError("m and n must be fp32")
-    _check_bias(bias, base_out, "dora_compose_fwd")
+    _like(base_out, where, lora_out=lora_out, y=y)
+    _vec_f32(d_out, where, m=m, n=n)
+    _check_bias(bias, base_out, where)
+    _dense_cuda(base_out, lora_out, m, n, y, bias)
     if y is None:
         y = torch.empty_like(base_out)
     head = (_ptr(base_out), _ptr(lora_out))
@@ -309,13 +352,13 @@ def dora_compose_fwd(base_out, lora_out, m, n, s: float, y=None, stream=None, bi
 def dora_compose_bwd(dy, base_out, lora_out, m, n, s: float, d_base=None, d_lora=None, d_m=None, workspace=None,
                      stream=None, bias=None):
     """(d_base, d_lora, d_m) of the compose with n held constant and the bias frozen."""
-    _dense_cuda(dy, base_out, lora_out, m, n, d_base, d_lora, d_m, workspace)
+    where = "dora_compose_bwd"
+    _acts2d(base_out, where)
     tokens, d_out = base_out.shape
-    if dy.shape != base_out.shape or lora_out.shape != base_out.shape:
-        raise ValueError("shape mismatch in dora_compose_bwd")
-    if m.dtype != torch.float32 or n.dtype != torch.float32:
-        raise TypeError("m and n must be fp32")
-    _check_bias(bias, base_out, "dora_compose_bwd")
+    _like(base_out, where, dy=dy, lora_out=lora_out, d_base=d_base, d_lora=d_lora)
+    _vec_f32(d_out, where, m=m, n=n, d_m=d_m)
+    _check_bias(bias, base_out, where)
+    _dense_cuda(dy, base_out, lora_out, m, n, d_base, d_lora, d_m, workspace, bias)
     if d_base is None:
         d_base = torch.empty_like(base_out)
     if d_lora is None:
@@ -339,15 +382,15 @@ def dora_compose_bwd(dy, base_out, lora_out, m, n, s: float, d_base=None, d_lora
 def dora_compose_bwd_noalloc(dy, base_out, lora_out, m, n, s: float, d_base, d_lora, d_m, stream=None, bias=None):
     """dora_compose_bwd into caller-provided outputs, with the library's own
     scratch instead of a workspace (nothing is allocated)."""
-    _dense_cuda(dy, base_out, lora_out, m, n, d_base, d_lora, d_m)
+    where = "dora_compose_bwd_noalloc"
+    if d_base is None or d_lora is None or d_m is None:
+        raise ValueError(f"{where}: d_base, d_lora and d_m are required (nothing is allocated)")
+    _acts2d(base_out, where)
     tokens, d_out = base_out.shape
-    if dy.shape != base_out.shape or lora_out.shape != base_out.shape:
-        raise ValueError("shape mismatch in dora_compose_bwd_noalloc")
-    if d_base.shape != base_out.shape or d_lora.shape != base_out.shape or d_m.shape != (d_out,):
-        raise ValueError("output shape mismatch in dora_compose_bwd_noalloc")
-    if m.dtype != torch.float32 or n.dtype != torch.float32 or d_m.dtype != torch.float32:
-        raise TypeError("m, n and d_m must be fp32")
-    _check_bias(bias, base_out, "dora_compose_bwd_noalloc")
+    _like(base_out, where, dy=dy, lora_out=lora_out, d_base=d_base, d_lora=d_lora)
+    _vec_f32(d_out, where, m=m, n=n, d_m=d_m)
+    _check_bias(bias, base_out, where)
+    _dense_cuda(dy, base_out, lora_out, m, n, d_base, d_lora, d_m, bias)
     head = (_ptr(dy), _ptr(base_out), _ptr(lora_out))
     tail = (_ptr(m), _ptr(n), float(s), tokens, d_out, _dt(base_out), _ptr(d_base), _ptr(d_lora), _ptr(d_m),
             _stream(stream))
@@ -365,20 +408,22 @@ def dora_fused_linear_fwd_workspace_size(tokens: int, r: int) -> int:
 
 def dora_fused_linear_fwd(x, W, A, B, m, n, s: float, bias=None, y=None, workspace=None, stream=None):
     """y = b + (m / n) * (x W^T + s * (x A^T) B^T), the compose fused into the GEMMs (bf16)."""
-    _dense_cuda(x, W, A, B, m, n, bias, y, workspace)
+    where = "dora_fused_linear_fwd"
+    if x.dim() != 2 or W.dim() != 2 or A.dim() != 2 or B.dim() != 2:
+        raise ValueError(f"{where}: x, W, A and B must be 2-D")
     T, d_in = x.shape
     d_out, r = W.shape[0], A.shape[0]
     if W.shape != (d_out, d_in) or A.shape != (r, d_in) or B.shape != (d_out, r):
         raise ValueError("shape mismatch in dora_fused_linear_fwd")
-    if m.shape != (d_out,) or n.shape != (d_out,):
-        raise ValueError("m and n must have shape (d_out,)")
-    if m.dtype != torch.float32 or n.dtype != torch.float32:
-        raise TypeError("m and n must be fp32")
+    _vec_f32(d_out, where, m=m, n=n)
     for t in (x, W, A, B):
         if t.dtype != torch.bfloat16:
             raise TypeError("x, W, A and B must be bf16")
     if bias is not None and (bias.shape != (d_out,) or bias.dtype != torch.bfloat16):
         raise ValueError("bias must be bf16 of shape (d_out,)")
+    if y is not None and (tuple(y.shape) != (T, d_out) or y.dtype != torch.bfloat16):
+        raise ValueError(f"{where}: y must be bf16 of shape ({T}, {d_out})")
+    _dense_cuda(x, W, A, B, m, n, bias, y, workspace)
     if y is None:
         y = torch.empty(T, d_out, dtype=torch.bfloat16, device=x.device)
     need = dora_fused_linear_fwd_workspace_size(T, r)
@@ -398,7 +443,9 @@ def dora_factored_norm_bwd_workspace_size(d_out: int, d_in: int, r: int) -> int:
 
 def dora_factored_norm_bwd(W, A, B, s: float, n, d_n, dA=None, dB=None, workspace=None, stream=None):
     """(dA, dB): gradients of n_i = ||W_i + s B_i A|| into A and B (fp32), given d_n = dL/dn."""
-    _dense_cuda(W, A, B, n, d_n, dA, dB, workspace)
+    where = "dora_factored_norm_bwd"
+    if W.dim() != 2 or A.dim() != 2 or B.dim() != 2:
+        raise ValueError(f"{where}: W, A and B must be 2-D")
     d_out, d_in = W.shape
     r = A.shape[0]
     if A.shape != (r, d_in) or B.shape != (d_out, r) or n.shape != (d_out,) or d_n.shape != (d_out,):
@@ -406,8 +453,11 @@ def dora_factored_norm_bwd(W, A, B, s: float, n, d_n, dA=None, dB=None, workspac
     for t in (W, A, B):
         if t.dtype != torch.bfloat16:
             raise TypeError("W, A and B must be bf16")
-    if n.dtype != torch.float32 or d_n.dtype != torch.float32:
-        raise TypeError("n and d_n must be fp32")
+    _vec_f32(d_out, where, n=n, d_n=d_n)
+    for name, t, shp in (("dA", dA, (r, d_in)), ("dB", dB, (d_out, r))):
+        if t is not None and (tuple(t.shape) != shp or t.dtype != torch.float32):
+            raise ValueError(f"{where}: {name} must be fp32 of shape {shp}")
+    _dense_cuda(W, A, B, n, d_n, dA, dB, workspace)
     if dA is None:
         dA = torch.empty(r, d_in, dtype=torch.float32, device=W.device)
     if dB is None:

@@ -211,6 +211,9 @@ DORA_API int dora_compose_bwd_bias(const void* dy, const void* base_out, const v
  * cudaMalloc, cudaFree or allocating library routine is called.  The first
  * call on a device looks the array's device address up (cudaGetSymbolAddress)
  * with that device current; make that first call before any stream capture.
+ * The address is kept per device and per CUDA context: after the context is
+ * destroyed and created again (cudaDeviceReset), the next call looks it up
+ * afresh, so make that call before any capture too.
  * Nothing is cleared before a call either: the arrival counters in the array
  * carry a per-call tag, so whatever they hold is ignored, and the array
  * keeps the last call's contents.  All calls on a device

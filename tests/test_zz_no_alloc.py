@@ -13,6 +13,7 @@ import torch
 from factored_weight_norm_b200 import dora as D
 from factored_weight_norm_b200 import workloads as wlmod
 from tests import parity as P
+import oracle
 
 pytestmark = pytest.mark.gpu
 MAX_D_OUT = 32768  # DORA_NOALLOC_MAX_D_OUT in include/dora.h
@@ -31,15 +32,18 @@ def _inputs(T, d_out, dtype):
     return dy, base, lora, m.contiguous(), n, wl.s
 
 
-def _noalloc(dy, base, lora, m, n, s, d_base, d_lora, d_m):
+def _noalloc(dy, base, lora, m, n, s, d_base, d_lora, d_m, bias=None):
     T, d_out = base.shape
     d_base.fill_(float("nan"))
     d_lora.fill_(float("nan"))
     d_m.fill_(float("nan"))
-    st = D.lib().dora_compose_bwd_noalloc(
-        _ptr(dy), _ptr(base), _ptr(lora), _ptr(m), _ptr(n), s, T, d_out,
-        D.DORA_BF16 if base.dtype == torch.bfloat16 else D.DORA_F32,
-        _ptr(d_base), _ptr(d_lora), _ptr(d_m), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    head = (_ptr(dy), _ptr(base), _ptr(lora))
+    tail = (_ptr(m), _ptr(n), s, T, d_out, D.DORA_BF16 if base.dtype == torch.bfloat16 else D.DORA_F32,
+            _ptr(d_base), _ptr(d_lora), _ptr(d_m), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    if bias is None:
+        st = D.lib().dora_compose_bwd_noalloc(*head, *tail)
+    else:
+        st = D.lib().dora_compose_bwd_noalloc_bias(*head, _ptr(bias), *tail)
     assert st == D.DORA_OK, D.status_string(st)
     return d_base, d_lora, d_m
 
@@ -79,3 +83,28 @@ def test_noalloc_f32_scalar_vectors_at_the_largest_width():
     torch.cuda.synchronize()
     for g, r, name in zip(got, ref, ("d_base", "d_lora", "d_m")):
         P.assert_act_close(g, P.f64(r), name)
+
+
+@pytest.mark.parametrize("dtype,d_out,with_bias", [("bf16", 1024, False), ("f32", 998, True)])
+def test_noalloc_against_the_oracle_twice(dtype, d_out, with_bias):
+    # the fp64 oracle's compose backward directly, so that a fault shared by
+    # both CUDA entry points cannot pass; fp32 with d_out not a multiple of 4
+    # runs one element per vector, with a bias
+    T = 96
+    dy, base, lora, m, n, s = _inputs(T, d_out, dtype)
+    bias = None
+    b64 = None
+    if with_bias:
+        g = torch.Generator(device="cpu").manual_seed(5)
+        bias = (0.5 * torch.randn(d_out, generator=g)).to(base.dtype).cuda()
+        base = (base + bias).contiguous()
+        b64 = P.f64(bias)
+    ref = oracle.compose_backward(P.f64(dy), P.f64(base), P.f64(lora), P.f64(m), P.f64(n), s, bias=b64)
+    outs = (torch.empty_like(base), torch.empty_like(base), torch.empty(d_out, device="cuda"))
+    for _ in range(2):
+        got = _noalloc(dy, base, lora, m, n, s, *outs, bias=bias)
+        torch.cuda.synchronize()
+        for gt, rf, name in zip(got, ref, ("d_base", "d_lora", "d_m")):
+            if name != "d_m" and base.dtype == torch.bfloat16:
+                rf = P.bf16_round(rf)
+            P.assert_act_close(gt, rf, name)
