@@ -9,7 +9,6 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
-#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <vector>
@@ -23,8 +22,6 @@
 #include "norm_bwd.cuh"
 #include "norm_simt.cuh"
 #include "norm_tc.cuh"
-#include "norm_pair.cuh"
-#include "gram_cluster.cuh"
 #include "norm_batched.cuh"
 
 namespace dora {
@@ -82,7 +79,6 @@ struct DeviceInfo {
   int smem_optin = 0;
   int* status = nullptr;
   int pair_clusters = 0;  // co-resident 2-CTA clusters of linear_pair_kernel
-  int norm_clusters = 0;  // co-resident 2-CTA clusters of norm_pair_kernel
 };
 
 std::mutex g_mu;
@@ -110,9 +106,6 @@ int device_info(DeviceInfo** out) {
       return DORA_ERR_CUDA;
     if (cudaFuncSetAttribute(gram_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin) != cudaSuccess)
       return DORA_ERR_CUDA;
-    if (cudaFuncSetAttribute(gram_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kGcSmem)) != cudaSuccess)
-      return DORA_ERR_CUDA;
     if (cudaFuncSetAttribute(norm_batched_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin) !=
             cudaSuccess ||
         cudaFuncSetAttribute(gram_batched_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin) !=
@@ -120,26 +113,8 @@ int device_info(DeviceInfo** out) {
       return DORA_ERR_CUDA;
     if (pair_attrs(linear_pair_kernel<false, false>, d.smem_optin) ||
         pair_attrs(linear_pair_kernel<false, true>, d.smem_optin) ||
-        pair_attrs(linear_pair_kernel<true, true>, d.smem_optin) || pair_attrs(norm_pair_kernel, d.smem_optin))
+        pair_attrs(linear_pair_kernel<true, true>, d.smem_optin))
       return DORA_ERR_CUDA;
-    {
-      // every norm_pair_kernel configuration takes more than half of an SM's
-      // shared memory, so one pair per two SMs; counted at the largest size
-      cudaLaunchConfig_t occ{};
-      cudaLaunchAttribute cl[1];
-      cl[0].id = cudaLaunchAttributeClusterDimension;
-      cl[0].val.clusterDim.x = 2;
-      cl[0].val.clusterDim.y = 1;
-      cl[0].val.clusterDim.z = 1;
-      occ.gridDim = dim3(2 * (d.num_sms / 2));
-      occ.blockDim = dim3(kPnThreads);
-      occ.dynamicSmemBytes = d.smem_optin;
-      occ.attrs = cl;
-      occ.numAttrs = 1;
-      if (cudaOccupancyMaxActiveClusters(&d.norm_clusters, norm_pair_kernel, &occ) != cudaSuccess ||
-          d.norm_clusters < 1)
-        return DORA_ERR_CUDA;
-    }
     {
       cudaLaunchConfig_t occ{};
       cudaLaunchAttribute cl[1];
@@ -230,15 +205,12 @@ TcPlan plan_tc(int64_t d_out, int64_t d_in, int64_t r) {
   size_t off = 0;
   p.off_gs = off;
   off = align_up(off + static_cast<size_t>(r) * r * 2, 1024);
-  p.off_gp = off;  // (G' is reduced inside its cluster: no fp32 Gram partials in the workspace)
+  p.off_gp = off;
+  off = align_up(off + static_cast<size_t>(p.gram_splits_max) * p.gram_tiles * kBoxRows * kBoxRows * 4, 256);
   p.off_part = off;
-  // per-(row, segment) partials of the pair kernel: (pairs + pair tiles) x
-  // 256 rows, with its chunks of at most kPnMaxChunk columns
-  const long long pair_tiles = cdiv(d_out, kPnTileRows) * cdiv(r, kPnMaxChunk);
-  off = align_up(off + static_cast<size_t>(kMaxGrid / 2 + pair_tiles) * kPnTileRows * 4, 256);
+  off = align_up(off + static_cast<size_t>(kMaxGrid + p.m_tiles * p.n_chunks) * kBM * 4, 256);
   p.off_cnt = off;
-  // 64-bit tagged counters, two per pair M tile, the start ticket, the exit count
-  off = align_up(off + static_cast<size_t>(2 * cdiv(d_out, kPnTileRows) + 2) * 8, 256);
+  off = align_up(off + static_cast<size_t>(p.m_tiles) * 4, 256);
   p.total = off;
   return p;
 }
@@ -273,140 +245,85 @@ long long bwd_chunks(long long strips, long long slots, long long tokens, long l
   return std::max<long long>(1, std::min<long long>(k, k_max));
 }
 
-// The pair kernel's chunking of r: at most kPnMaxChunk columns per chunk,
-// equal chunk widths (a multiple of 16, rows past r read as zeros), each
-// chunk one MMA piece of up to 256 columns plus the rest; as many ring stages
-// as fit.
-struct PairPlan {
-  int n_chunks, chunk_n, h0, h1, pm_tiles, tiles, units, stages, b_boxes, b_per_item, b_items;
-  uint32_t stage_bytes;
-};
-
-PairPlan plan_pair(int64_t d_out, int64_t d_in, int64_t r, int smem_optin) {
-  PairPlan q{};
-  q.n_chunks = static_cast<int>(cdiv(r, kPnMaxChunk));
-  q.chunk_n = static_cast<int>(align_up(static_cast<size_t>(cdiv(r, q.n_chunks)), 16));
-  const int n0 = std::min(256, q.chunk_n);
-  q.h0 = n0 / 2;
-  q.h1 = (q.chunk_n - n0) / 2;
-  q.pm_tiles = static_cast<int>(cdiv(d_out, kPnTileRows));
-  q.tiles = q.pm_tiles * q.n_chunks;
-  const int kb_total = static_cast<int>(cdiv(d_in, kBK) + cdiv(r, kBK));
-  q.units = q.tiles * kb_total;
-  q.stage_bytes = kPnWBytes + static_cast<uint32_t>(q.h0 + q.h1) * 128u;
-  const long long room = static_cast<long long>(smem_optin) - kPnSmemFixed;
-  q.stages = static_cast<int>(std::max<long long>(0, std::min<long long>(kPnMaxStages, room / q.stage_bytes)));
-  // a segment's B rows travel as ring items of as many 64-column boxes as a slot holds
-  q.b_boxes = static_cast<int>(cdiv(q.chunk_n, kBK));
-  q.b_per_item = static_cast<int>(q.stage_bytes / kBoxBytes);
-  q.b_items = static_cast<int>(cdiv(q.b_boxes, q.b_per_item));
-  return q;
-}
-
 int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_t d_in, int64_t r, float s,
               float* n_out, void* ws, cudaStream_t st, DeviceInfo* dev, bool squared) {
   const TcPlan p = plan_tc(d_out, d_in, r);
-  const PairPlan q = plan_pair(d_out, d_in, r, dev->smem_optin);
-  if (q.stages < 2) return DORA_ERR_UNSUPPORTED;
   uint8_t* w = static_cast<uint8_t*>(ws);
   __nv_bfloat16* Gs = reinterpret_cast<__nv_bfloat16*>(w + p.off_gs);
+  float* Gp = reinterpret_cast<float*>(w + p.off_gp);
   float* part = reinterpret_cast<float*>(w + p.off_part);
-  unsigned long long* cnt = reinterpret_cast<unsigned long long*>(w + p.off_cnt);
+  int* cnt = reinterpret_cast<int*>(w + p.off_cnt);
 
-  CUtensorMap tmA, tmW, tmB, tmA0, tmA1, tmG0, tmG1;
-  if (make_map(&tmA, A, r, d_in) || make_map(&tmW, W, d_out, d_in) || make_map(&tmB, B, d_out, r) ||
-      make_map(&tmA0, A, r, d_in, q.h0) || make_map(&tmG0, Gs, r, r, q.h0))
+  CUtensorMap tmW, tmA, tmB, tmG;
+  if (make_map(&tmW, W, d_out, d_in) || make_map(&tmA, A, r, d_in) || make_map(&tmB, B, d_out, r) ||
+      make_map(&tmG, Gs, r, r))
     return DORA_ERR_CUDA;
-  if (q.h1 > 0) {
-    if (make_map(&tmA1, A, r, d_in, q.h1) || make_map(&tmG1, Gs, r, r, q.h1)) return DORA_ERR_CUDA;
-  } else {
-    tmA1 = tmA0;
-    tmG1 = tmG0;
-  }
 
-  // 1) G' = (s/2) A A^T by clusters of kGcSplit CTAs (the upper-triangle
-  // tiles), 2) the pair GEMM, launched behind it with programmatic dependent
-  // launch: its CTAs take the SMs the Gram clusters leave free, and its
-  // producers wait for the Gram grid only before their first K-extension block.
-  const int nt = static_cast<int>(cdiv(r, kBM));
-  GramClusterArgs gca{};
-  gca.r = static_cast<int>(r);
-  gca.kb_main = p.kb_main;
-  gca.nt = nt;
-  gca.half_s = 0.5f * s;
-  gca.Gs = Gs;
-  gca.wait_limit = kWaitLimitCycles;
-  gca.status = dev->status;
-  cudaLaunchAttribute gat[1];
-  gat[0].id = cudaLaunchAttributeClusterDimension;
-  gat[0].val.clusterDim.x = kGcSplit;
-  gat[0].val.clusterDim.y = 1;
-  gat[0].val.clusterDim.z = 1;
-  cudaLaunchConfig_t gcfg{};
-  gcfg.stream = st;
-  gcfg.attrs = gat;
-  gcfg.numAttrs = 1;
-  gcfg.gridDim = dim3(static_cast<unsigned>(nt * (nt + 1) / 2 * kGcSplit));
-  gcfg.blockDim = dim3(kGcThreads);
-  gcfg.dynamicSmemBytes = kGcSmem;
-  if (cudaLaunchKernelEx(&gcfg, gram_cluster_kernel, tmA, gca) != cudaSuccess) return DORA_ERR_CUDA;
+  // 1) Gram partial tiles, 2) reduce to bf16 (s/2) G and zero the counters,
+  // 3) the persistent GEMM; 2) and 3) use programmatic dependent launch so
+  // they are scheduled while their predecessor still runs and wait for it
+  // only where they read its results.
+  GramArgs ga{};
+  ga.r = static_cast<int>(r);
+  ga.kb_main = p.kb_main;
+  ga.splits = std::max(1, std::min(p.gram_splits_max, dev->num_sms / p.gram_tiles));
+  ga.n_tiles = static_cast<int>(cdiv(r, kBoxRows));
+  ga.wait_limit = kWaitLimitCycles;
+  ga.partial = Gp;
+  ga.status = dev->status;
+  ga.n_ctas1 = p.gram_tiles * ga.splits;
+  const size_t gram_smem = kGramStages * kGramStageBytes + (2 * kGramStages + 1) * 8 + 16 + 1024;
+  gram_tc_kernel<<<p.gram_tiles * ga.splits, kNormThreads, gram_smem, st>>>(tmA, tmA, tmA, tmA, ga);
+  if (launch_error()) return DORA_ERR_CUDA;
 
-  cudaLaunchAttribute at[2];
-  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  at[0].val.programmaticStreamSerializationAllowed = 1;
-  at[1].id = cudaLaunchAttributeClusterDimension;
-  at[1].val.clusterDim.x = 2;
-  at[1].val.clusterDim.y = 1;
-  at[1].val.clusterDim.z = 1;
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg{};
   cfg.stream = st;
-  cfg.attrs = at;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
 
-  const int P = std::max(1, std::min({dev->norm_clusters, dev->num_sms / 2, q.units, kMaxGrid / 2}));
-  PairNormArgs pa{};
-  pa.d_out = static_cast<int>(d_out);
-  pa.d_in = static_cast<int>(d_in);
-  pa.r = static_cast<int>(r);
-  pa.n_chunks = q.n_chunks;
-  pa.chunk_n = q.chunk_n;
-  pa.kb_main = p.kb_main;
-  pa.kb_total = p.kb_total;
-  pa.pm_tiles = q.pm_tiles;
-  pa.tiles = q.tiles;
-  pa.units = q.units;
-  {
-    // the Gram clusters hold one SM per CTA for about one unit of GEMM time
-    // per K block of their split; pairs that start after them get that much
-    // less, so that all end together
-    const int gram_sms = std::min(dev->num_sms, nt * (nt + 1) / 2 * kGcSplit);
-    pa.early = std::max(0, std::min(P, (dev->num_sms - gram_sms) / 2));
-    const double d = static_cast<double>(cdiv(p.kb_main, kGcSplit));
-    const double f = (q.units + static_cast<double>(P - pa.early) * d) / P;
-    pa.w_early = std::max<long long>(1, std::llround(16.0 * f));
-    pa.w_late = pa.early < P ? std::max<long long>(0, std::llround(16.0 * (f - d))) : pa.w_early;
-  }
-  pa.stages = q.stages;
-  pa.stage_bytes = q.stage_bytes;
-  pa.B = static_cast<const __nv_bfloat16*>(B);
-  pa.b_boxes = q.b_boxes;
-  pa.b_per_item = q.b_per_item;
-  pa.b_items = q.b_items;
-  pa.h0 = q.h0;
-  pa.h1 = q.h1;
-  pa.two_s = 2.0f * s;
-  pa.wait_limit = kWaitLimitCycles;
-  pa.tag = (next_bwd_epoch() & ((1ull << 40) - 1)) << kPnTagShift;
-  pa.partials = part;
-  pa.counters = cnt;
-  pa.n_out = n_out;
-  pa.status = dev->status;
-  pa.squared = squared ? 1 : 0;
-  cfg.numAttrs = 2;
-  cfg.gridDim = dim3(2 * P);
-  cfg.blockDim = dim3(kPnThreads);
-  cfg.dynamicSmemBytes = static_cast<size_t>(q.stages) * q.stage_bytes + kPnSmemFixed;
-  if (cudaLaunchKernelEx(&cfg, norm_pair_kernel, tmW, tmB, tmA0, tmA1, tmG0, tmG1, pa) != cudaSuccess)
+  const long long rr = static_cast<long long>(r) * r;
+  const unsigned red_grid = static_cast<unsigned>(
+      std::max<long long>(cdiv(p.m_tiles, 256), std::min<long long>(cdiv(rr, 1024), 4 * dev->num_sms)));
+  cfg.gridDim = dim3(red_grid);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  if (cudaLaunchKernelEx(&cfg, gram_reduce_kernel, static_cast<const float*>(Gp), ga.splits, static_cast<int>(r),
+                         0.5f * s, Gs, cnt, p.m_tiles, static_cast<int>(red_grid), static_cast<const float*>(nullptr), 0,
+                         0.f, static_cast<__nv_bfloat16*>(nullptr)) != cudaSuccess)
     return DORA_ERR_CUDA;
+
+  NormArgs na{};
+  na.d_out = static_cast<int>(d_out);
+  na.d_in = static_cast<int>(d_in);
+  na.r = static_cast<int>(r);
+  na.m_tiles = p.m_tiles;
+  na.n_chunks = p.n_chunks;
+  na.chunk_n = p.chunk_n;
+  na.kb_main = p.kb_main;
+  na.kb_total = p.kb_total;
+  na.units = p.units;
+  na.stage_bytes = static_cast<uint32_t>(kBoxBytes * (1 + cdiv(p.chunk_n, kBoxRows)));
+  na.stages = static_cast<int>(
+      std::min<size_t>(kMaxStages, (dev->smem_optin - kNormTcSmemFixed) / (na.stage_bytes + 16)));
+  if (na.stages < 2) return DORA_ERR_UNSUPPORTED;
+  uint32_t cols = 32;
+  while (cols < static_cast<uint32_t>(p.chunk_n)) cols <<= 1;
+  na.tmem_cols = cols;
+  na.two_s = 2.0f * s;
+  na.wait_limit = kWaitLimitCycles;
+  na.partials = part;
+  na.counters = cnt;
+  na.n_out = n_out;
+  na.status = dev->status;
+  na.squared = squared ? 1 : 0;
+  const int grid = static_cast<int>(std::min<long long>({static_cast<long long>(dev->num_sms), p.units, kMaxGrid}));
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kNormTcThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(na.stages) * (na.stage_bytes + 16) + kNormTcSmemFixed;
+  if (cudaLaunchKernelEx(&cfg, norm_tc_kernel, tmW, tmA, tmB, tmG, na) != cudaSuccess) return DORA_ERR_CUDA;
   return launch_error();
 }
 

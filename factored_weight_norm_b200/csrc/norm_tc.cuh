@@ -742,10 +742,7 @@ __global__ void __launch_bounds__(kNormThreads, 1)
 // bf16 G' the norm kernel's K extension reads; also zeroes the norm kernel's
 // tile counters.  CTAs from `g1` on reduce a second product the same way
 // (`partial2`, `splits2`, `scale2`, `Gs2`; a Gram launch of two products).
-// 64 registers a thread at most (__launch_bounds__(256, 4)): a CTA of it then
-// leaves room in an SM's register file for a CTA of the GEMM launched behind
-// it, which can start its streaming while the reduction still runs.
-__global__ void __launch_bounds__(256, 4) gram_reduce_kernel(const float* __restrict__ partial, int splits, int r, float half_s,
+__global__ void gram_reduce_kernel(const float* __restrict__ partial, int splits, int r, float half_s,
                                    __nv_bfloat16* __restrict__ Gs, int* counters, int n_counters, int g1,
                                    const float* __restrict__ partial2, int splits2, float scale2,
                                    __nv_bfloat16* __restrict__ Gs2) {
@@ -763,9 +760,9 @@ __global__ void __launch_bounds__(256, 4) gram_reduce_kernel(const float* __rest
   const long long total = static_cast<long long>(r) * r;
   const int nt = (r + kBoxRows - 1) / kBoxRows;
   const long long split_stride = static_cast<long long>(nt) * nt * kBoxRows * kBoxRows;
-  // four elements per thread and four splits per round: 16 independent loads
+  // four elements per thread and eight splits per round: 32 independent loads
   // in flight; each element still adds its splits in increasing order
-  constexpr int kE = 4, kS = 4;
+  constexpr int kE = 4, kS = 8;
   const long long step = static_cast<long long>(gx) * blockDim.x;
   for (long long base = bx * static_cast<long long>(blockDim.x) + threadIdx.x; base < total;
        base += kE * step) {
