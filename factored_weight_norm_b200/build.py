@@ -19,7 +19,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libdora.so")
 SOURCES = [os.path.join(CSRC, "dora_api.cu")]
 DEPS = SOURCES + [
-    os.path.join(CSRC, f) for f in ("sm100_ptx.cuh", "norm_tc.cuh", "norm_batched.cuh", "norm_simt.cuh", "compose.cuh", "linear_tc.cuh", "norm_bwd.cuh")
+    os.path.join(CSRC, f) for f in ("sm100_ptx.cuh", "norm_tc.cuh", "gram_cluster.cuh", "norm_batched.cuh", "norm_simt.cuh", "compose.cuh", "linear_tc.cuh", "norm_bwd.cuh")
 ] + [os.path.join(ROOT, "include", "dora.h")]
 
 NVCC_FLAGS = [

@@ -9,6 +9,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <vector>
@@ -22,6 +23,7 @@
 #include "norm_bwd.cuh"
 #include "norm_simt.cuh"
 #include "norm_tc.cuh"
+#include "gram_cluster.cuh"
 #include "norm_batched.cuh"
 
 namespace dora {
@@ -66,6 +68,7 @@ int pair_attrs(K kernel, int smem_optin) {
 }
 constexpr int kMaxGrid = 1024;                         // bound on the persistent grid
 constexpr int kMaxGramSplits = 32;
+constexpr int kGramBlocksPerSplit = 32;                // K blocks a Gram CTA of the norm takes, about
 constexpr int kMaxBwdChunks = 64;
 constexpr int kMaxDevices = 64;
 constexpr int64_t kMaxRank = 4096;
@@ -90,6 +93,16 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 EncodeTiledFn g_encode = nullptr;
 
 // Per-device set-up, done once with that device current.
+template <typename K>
+int gram_cluster_attrs(K kernel) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kGcSmem)) !=
+                 cudaSuccess ||
+             cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                  cudaSharedmemCarveoutMaxShared) != cudaSuccess
+             ? DORA_ERR_CUDA
+             : DORA_OK;
+}
+
 int device_info(DeviceInfo** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DORA_ERR_CUDA;
@@ -105,6 +118,20 @@ int device_info(DeviceInfo** out) {
     if (cudaFuncSetAttribute(norm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin) != cudaSuccess)
       return DORA_ERR_CUDA;
     if (cudaFuncSetAttribute(gram_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin) != cudaSuccess)
+      return DORA_ERR_CUDA;
+    // Kernels that run beside the first CTAs of a GEMM launched behind them
+    // ask for the largest shared-memory carveout: an SM configured for a
+    // small one (the default for a kernel with little shared memory) takes no
+    // GEMM CTA until it drains.
+    if (cudaFuncSetAttribute(gram_reduce_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess ||
+        cudaFuncSetAttribute(gram_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess ||
+        cudaFuncSetAttribute(norm_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+      return DORA_ERR_CUDA;
+    if (gram_cluster_attrs(gram_cluster_kernel<1>) || gram_cluster_attrs(gram_cluster_kernel<2>) ||
+        gram_cluster_attrs(gram_cluster_kernel<4>) || gram_cluster_attrs(gram_cluster_kernel<8>))
       return DORA_ERR_CUDA;
     if (cudaFuncSetAttribute(norm_batched_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin) !=
             cudaSuccess ||
@@ -186,8 +213,7 @@ void launch_compose_bwd(dim3 grid, cudaStream_t st, const void* dy, const void* 
 struct TcPlan {
   int m_tiles, n_chunks, chunk_n, kb_main, kb_ext, kb_total;
   long long units;
-  int gram_tiles, gram_splits_max;
-  size_t off_gs, off_gp, off_part, off_cnt, total;
+  size_t off_gs, off_part, off_cnt, total;
 };
 
 TcPlan plan_tc(int64_t d_out, int64_t d_in, int64_t r) {
@@ -199,14 +225,10 @@ TcPlan plan_tc(int64_t d_out, int64_t d_in, int64_t r) {
   p.kb_ext = static_cast<int>(cdiv(r, kBK));
   p.kb_total = p.kb_main + p.kb_ext;
   p.units = static_cast<long long>(p.m_tiles) * p.n_chunks * p.kb_total;
-  const int nt = static_cast<int>(cdiv(r, kBoxRows));
-  p.gram_tiles = nt * nt;
-  p.gram_splits_max = std::max(1, std::min({kMaxGramSplits, 160 / p.gram_tiles, p.kb_main}));
   size_t off = 0;
   p.off_gs = off;
   off = align_up(off + static_cast<size_t>(r) * r * 2, 1024);
-  p.off_gp = off;
-  off = align_up(off + static_cast<size_t>(p.gram_splits_max) * p.gram_tiles * kBoxRows * kBoxRows * 4, 256);
+  // (the Gram clusters keep their K-split partials in shared memory)
   p.off_part = off;
   off = align_up(off + static_cast<size_t>(kMaxGrid + p.m_tiles * p.n_chunks) * kBM * 4, 256);
   p.off_cnt = off;
@@ -248,9 +270,9 @@ long long bwd_chunks(long long strips, long long slots, long long tokens, long l
 int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_t d_in, int64_t r, float s,
               float* n_out, void* ws, cudaStream_t st, DeviceInfo* dev, bool squared) {
   const TcPlan p = plan_tc(d_out, d_in, r);
+  if (p.units > (1ll << 30)) return DORA_ERR_UNSUPPORTED;  // unit indices are 32-bit in the kernel
   uint8_t* w = static_cast<uint8_t*>(ws);
   __nv_bfloat16* Gs = reinterpret_cast<__nv_bfloat16*>(w + p.off_gs);
-  float* Gp = reinterpret_cast<float*>(w + p.off_gp);
   float* part = reinterpret_cast<float*>(w + p.off_part);
   int* cnt = reinterpret_cast<int*>(w + p.off_cnt);
 
@@ -259,22 +281,52 @@ int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_
       make_map(&tmG, Gs, r, r))
     return DORA_ERR_CUDA;
 
-  // 1) Gram partial tiles, 2) reduce to bf16 (s/2) G and zero the counters,
-  // 3) the persistent GEMM; 2) and 3) use programmatic dependent launch so
-  // they are scheduled while their predecessor still runs and wait for it
-  // only where they read its results.
-  GramArgs ga{};
-  ga.r = static_cast<int>(r);
-  ga.kb_main = p.kb_main;
-  ga.splits = std::max(1, std::min(p.gram_splits_max, dev->num_sms / p.gram_tiles));
-  ga.n_tiles = static_cast<int>(cdiv(r, kBoxRows));
-  ga.wait_limit = kWaitLimitCycles;
-  ga.partial = Gp;
-  ga.status = dev->status;
-  ga.n_ctas1 = p.gram_tiles * ga.splits;
-  const size_t gram_smem = kGramStages * kGramStageBytes + (2 * kGramStages + 1) * 8 + 16 + 1024;
-  gram_tc_kernel<<<p.gram_tiles * ga.splits, kNormThreads, gram_smem, st>>>(tmA, tmA, tmA, tmA, ga);
-  if (launch_error()) return DORA_ERR_CUDA;
+  // 1) G' = (s/2) A A^T: one cluster of `splits` CTAs per tile on or above
+  // the diagonal, each CTA a K split, summed inside the cluster; the launch
+  // also zeroes the GEMM's tile counters.  2) The persistent GEMM behind it
+  // with programmatic dependent launch: its CTAs start on the SMs the Gram
+  // clusters leave free, meet G' only at the ends of their ranges and wait
+  // for the Gram launch only there.
+  const int nt = static_cast<int>(cdiv(r, kBoxRows));
+  const int up_tiles = nt * (nt + 1) / 2;
+  // about kGramBlocksPerSplit K blocks per CTA, on at most a third of the
+  // SMs; a power of two up to 8 (the cluster size)
+  int splits = 1;
+  while (splits < 8 && splits * kGramBlocksPerSplit < p.kb_main && 2 * splits <= p.kb_main &&
+         up_tiles * 2 * splits <= std::max(1, dev->num_sms / 3))
+    splits *= 2;
+  {
+    GramClusterArgs gca{};
+    gca.r = static_cast<int>(r);
+    gca.kb_main = p.kb_main;
+    gca.nt = nt;
+    gca.half_s = 0.5f * s;
+    gca.Gs = Gs;
+    gca.wait_limit = kWaitLimitCycles;
+    gca.status = dev->status;
+    gca.zero_cnt = cnt;
+    gca.n_zero = p.m_tiles;
+    cudaLaunchAttribute gat[1];
+    gat[0].id = cudaLaunchAttributeClusterDimension;
+    gat[0].val.clusterDim.x = static_cast<unsigned>(splits);
+    gat[0].val.clusterDim.y = 1;
+    gat[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t gcfg{};
+    gcfg.stream = st;
+    gcfg.attrs = gat;
+    gcfg.numAttrs = 1;
+    gcfg.gridDim = dim3(static_cast<unsigned>(up_tiles * splits));
+    gcfg.blockDim = dim3(kGcThreads);
+    gcfg.dynamicSmemBytes = kGcSmem;
+    cudaError_t e = cudaSuccess;
+    switch (splits) {
+      case 1: e = cudaLaunchKernelEx(&gcfg, gram_cluster_kernel<1>, tmA, gca); break;
+      case 2: e = cudaLaunchKernelEx(&gcfg, gram_cluster_kernel<2>, tmA, gca); break;
+      case 4: e = cudaLaunchKernelEx(&gcfg, gram_cluster_kernel<4>, tmA, gca); break;
+      default: e = cudaLaunchKernelEx(&gcfg, gram_cluster_kernel<8>, tmA, gca); break;
+    }
+    if (e != cudaSuccess) return DORA_ERR_CUDA;
+  }
 
   cudaLaunchAttribute pdl[1];
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -283,17 +335,6 @@ int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_
   cfg.stream = st;
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
-
-  const long long rr = static_cast<long long>(r) * r;
-  const unsigned red_grid = static_cast<unsigned>(
-      std::max<long long>(cdiv(p.m_tiles, 256), std::min<long long>(cdiv(rr, 1024), 4 * dev->num_sms)));
-  cfg.gridDim = dim3(red_grid);
-  cfg.blockDim = dim3(256);
-  cfg.dynamicSmemBytes = 0;
-  if (cudaLaunchKernelEx(&cfg, gram_reduce_kernel, static_cast<const float*>(Gp), ga.splits, static_cast<int>(r),
-                         0.5f * s, Gs, cnt, p.m_tiles, static_cast<int>(red_grid), static_cast<const float*>(nullptr), 0,
-                         0.f, static_cast<__nv_bfloat16*>(nullptr)) != cudaSuccess)
-    return DORA_ERR_CUDA;
 
   NormArgs na{};
   na.d_out = static_cast<int>(d_out);
@@ -305,11 +346,13 @@ int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_
   na.kb_main = p.kb_main;
   na.kb_total = p.kb_total;
   na.units = p.units;
+  const int grid = static_cast<int>(std::min<long long>({static_cast<long long>(dev->num_sms), p.units, kMaxGrid}));
+  const size_t smem_fixed = kNormTcSmemFixed + static_cast<size_t>(grid + 1) * 4;  // + the range-start table
   na.stage_bytes = static_cast<uint32_t>(kBoxBytes * (1 + cdiv(p.chunk_n, kBoxRows)));
-  na.stages = static_cast<int>(
-      std::min<size_t>(kMaxStages, (dev->smem_optin - kNormTcSmemFixed) / (na.stage_bytes + 16)));
+  na.stages = static_cast<int>(std::min<size_t>(kMaxStages, (dev->smem_optin - smem_fixed) / (na.stage_bytes + 16)));
   if (na.stages < 2) return DORA_ERR_UNSUPPORTED;
-  uint32_t cols = 32;
+  // a power of two of at least 64 columns: the epilogue reads V 64 columns at a time
+  uint32_t cols = 64;
   while (cols < static_cast<uint32_t>(p.chunk_n)) cols <<= 1;
   na.tmem_cols = cols;
   na.two_s = 2.0f * s;
@@ -319,10 +362,28 @@ int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_
   na.n_out = n_out;
   na.status = dev->status;
   na.squared = squared ? 1 : 0;
-  const int grid = static_cast<int>(std::min<long long>({static_cast<long long>(dev->num_sms), p.units, kMaxGrid}));
+  {
+    // The Gram CTAs hold one SM each (their shared memory): that many CTAs of
+    // the GEMM start late and get that much less, so that all end together.
+    // Start delay and GEMM unit time from traces of these kernels on B200
+    // (8192 x 8192, r = 64 and 384): a Gram CTA takes about 3 us plus
+    // 0.43 us per K block of its split, plus about 5 us to sum and mirror
+    // off-diagonal tiles; a GEMM unit about 0.18 us plus 0.01 us per KB of its
+    // ring stage.  A late CTA that ends early costs the grid a little; one
+    // that ends late costs the whole gap, so the delay is taken 10% long.
+    const int gram_sms = std::min(dev->num_sms, up_tiles * splits);
+    const int late = grid > gram_sms ? gram_sms : 0;
+    const double gram_us = 3.0 + 0.43 * static_cast<double>(cdiv(p.kb_main, splits)) + (nt > 1 ? 5.0 : 1.0);
+    const double unit_us = 0.18 + 0.01 * (static_cast<double>(na.stage_bytes) / 1024.0);
+    const double delay = 1.1 * gram_us / unit_us;
+    const double f = (static_cast<double>(p.units) + late * delay) / grid;
+    na.early = grid - late;
+    na.w_early = std::max<long long>(1, std::llround(16.0 * f));
+    na.w_late = late > 0 ? std::max<long long>(0, std::llround(16.0 * (f - delay))) : na.w_early;
+  }
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kNormTcThreads);
-  cfg.dynamicSmemBytes = static_cast<size_t>(na.stages) * (na.stage_bytes + 16) + kNormTcSmemFixed;
+  cfg.dynamicSmemBytes = static_cast<size_t>(na.stages) * (na.stage_bytes + 16) + smem_fixed;
   if (cudaLaunchKernelEx(&cfg, norm_tc_kernel, tmW, tmA, tmB, tmG, na) != cudaSuccess) return DORA_ERR_CUDA;
   return launch_error();
 }
@@ -961,7 +1022,8 @@ int dora_factored_norm_bwd(const void* W, const void* A, const void* B, float s,
   ga.splits = std::max(1, std::min({L.splits_max, (dev->num_sms / 2) / (L.nt * L.nt), kb_g}));
   ga.kb_main2 = kb_h;
   ga.splits2 = std::max(1, std::min({L.splits_max, (dev->num_sms / 2) / (L.nt * L.nt), kb_h}));
-  ga.n_ctas1 = L.nt * L.nt * ga.splits;
+  ga.upper = 1;  // G = A A^T is symmetric: its tiles on or above the diagonal only
+  ga.n_ctas1 = L.nt * (L.nt + 1) / 2 * ga.splits;
   ga.partial = part;
   ga.partial2 = part2;
   ga.wait_limit = kWaitLimitCycles;
@@ -980,7 +1042,7 @@ int dora_factored_norm_bwd(const void* W, const void* A, const void* B, float s,
     cfg.blockDim = dim3(256);
     if (cudaLaunchKernelEx(&cfg, gram_reduce_kernel, static_cast<const float*>(part), ga.splits, static_cast<int>(r), s,
                            sG, static_cast<int*>(nullptr), 0, g1, static_cast<const float*>(part2), ga.splits2, s,
-                           s2H) != cudaSuccess)
+                           s2H, 1) != cudaSuccess)
       return DORA_ERR_CUDA;
   }
 

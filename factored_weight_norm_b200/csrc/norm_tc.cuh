@@ -47,6 +47,7 @@ constexpr int kNormTcThreads = 256;
 // shared memory besides the stages: 1024-byte alignment slack, five single
 // mbarriers, the TMEM address and abort flag (16 bytes), the W^2 hand-off
 // (kBM floats); each stage adds its two mbarriers
+// (plus the table of the grid's G + 1 range starts, 4 bytes each)
 constexpr int kNormTcSmemFixed = 1024 + 5 * 8 + 16 + kBM * 4;
 constexpr int kMaxChunkN = 512;       // TMEM columns
 constexpr int kMaxStages = 8;
@@ -57,23 +58,46 @@ struct NormArgs {
   int d_out, d_in, r;
   int m_tiles, n_chunks, chunk_n, kb_main, kb_total;
   long long units;
+  // CTA c's unit range is [unit_start(c), unit_start(c + 1)): lengths in
+  // proportion to w_early for the first `early` CTAs and to w_late after (the
+  // CTAs that wait for the SMs the Gram launch holds)
+  int early;
+  long long w_early, w_late;
   int stages;
   uint32_t stage_bytes;   // W-side tile + N-side tiles (a multiple of kBoxBytes)
   uint32_t tmem_cols;
   float two_s;
   long long wait_limit;
   float* partials;        // [(gridDim.x + m_tiles * n_chunks) * 128]
-  int* counters;          // [m_tiles], zeroed by gram_reduce_kernel
+  int* counters;          // [m_tiles], zeroed by the Gram launch ahead of this one
   float* n_out;           // [d_out]
   int* status;
   int squared;            // 1: write n^2 as summed (a shard's partial), 0: sqrt(max(n^2, 0))
 };
 
-// Owner CTA of unit u when U units are split into G contiguous ranges
-// [floor(c U / G), floor((c + 1) U / G)).
-__host__ __device__ __forceinline__ int stream_k_owner(long long u, long long U, int G) {
-  return static_cast<int>(((u + 1) * static_cast<long long>(G) - 1) / U);
+// Weighted stream-K ranges: CTA c owns [unit_start(c), unit_start(c + 1)),
+// the cumulative weight of the CTAs before c scaled to the unit count.  The
+// kernel tabulates the starts in shared memory once; the lookups below run
+// on that table.
+__host__ __device__ __forceinline__ long long unit_cum(const NormArgs& a, int c) {
+  return a.w_early * (c < a.early ? c : a.early) + a.w_late * (c > a.early ? c - a.early : 0);
 }
+__host__ __device__ __forceinline__ long long unit_start(const NormArgs& a, int c, int G) {
+  return a.units * unit_cum(a, c) / unit_cum(a, G);
+}
+// Owner of unit u in the table `st` of G + 1 starts: the largest c with
+// st[c] <= u (an empty range never owns a unit, since the next range starts
+// where it does).
+__device__ __forceinline__ int unit_owner(const int* st, int u, int G) {
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (st[mid] <= u) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+__device__ __forceinline__ bool unit_range_nonempty(const int* st, int c) { return st[c + 1] > st[c]; }
 
 __device__ __forceinline__ void record_timeout(int* status, volatile int* abort_flag) {
   atomicExch(status, kStatusTimeout);
@@ -110,27 +134,51 @@ __device__ __forceinline__ uint32_t sw128_chunk(int row, int c) {
   return static_cast<uint32_t>(row * 128 + ((c ^ (row & 7)) << 4));
 }
 
-// Walks a CTA's contiguous range of (M tile, N chunk, K block) units in order.
-// Only the start needs a division; stepping is compare-and-increment, so the
-// single-thread producer and MMA loops spend a few instructions per unit.
+// Walks a CTA's range of (M tile, N chunk, K block) units.  A range [u0, u1)
+// that crosses a tile boundary is walked from its first boundary tb on,
+// [tb, u1), then [u0, tb): the part that ends with a tile's K-extension
+// blocks (the only reads of the Gram launch's G') comes last, so a CTA
+// seldom waits for that launch.  Only the starts need a division; stepping
+// is compare-and-increment, so the single-thread producer and MMA loops
+// spend a few instructions per unit.
 struct UnitIter {
   int tc, kb, mt, ch, c0, n_this, left;
+  int len2;               // units of the part walked second (0: no wrap)
+  long long wrap_to;      // its first unit
   bool seg_first;
 
-  __device__ __forceinline__ void start(const NormArgs& a, long long u_begin, long long u_end) {
-    tc = static_cast<int>(u_begin / a.kb_total);
-    kb = static_cast<int>(u_begin - static_cast<long long>(tc) * a.kb_total);
+  __device__ __forceinline__ void seek(const NormArgs& a, long long u) {
+    tc = static_cast<int>(u / a.kb_total);
+    kb = static_cast<int>(u - static_cast<long long>(tc) * a.kb_total);
     mt = tc / a.n_chunks;
     ch = tc - mt * a.n_chunks;
     c0 = ch * a.chunk_n;
     n_this = min(a.chunk_n, a.r - c0);
-    left = static_cast<int>(u_end - u_begin);
     seg_first = true;
   }
+  __device__ __forceinline__ void start(const NormArgs& a, long long u_begin, long long u_end) {
+    const long long tb = min(u_end, (u_begin + a.kb_total - 1) / a.kb_total * a.kb_total);
+    left = static_cast<int>(u_end - u_begin);
+    if (tb > u_begin && tb < u_end) {
+      len2 = static_cast<int>(tb - u_begin);
+      wrap_to = u_begin;
+      seek(a, tb);
+    } else {
+      len2 = 0;
+      wrap_to = 0;
+      seek(a, u_begin);
+    }
+  }
   __device__ __forceinline__ bool valid() const { return left > 0; }
-  __device__ __forceinline__ bool seg_last(const NormArgs& a) const { return left == 1 || kb == a.kb_total - 1; }
+  __device__ __forceinline__ bool seg_last(const NormArgs& a) const {
+    return left == 1 || kb == a.kb_total - 1 || (len2 > 0 && left == len2 + 1);
+  }
   __device__ __forceinline__ void next(const NormArgs& a) {
     --left;
+    if (len2 > 0 && left == len2) {
+      seek(a, wrap_to);
+      return;
+    }
     if (++kb == a.kb_total) {
       kb = 0;
       ++tc;
@@ -173,13 +221,14 @@ __global__ void __launch_bounds__(kNormTcThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(w2_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* w2 = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(w2_empty + 1) + 16);
+  int* starts = reinterpret_cast<int*>(w2 + kBM);  // [gridDim.x + 1] unit range starts
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const long long U = a.units;
   const int G = gridDim.x;
-  const long long u_begin = static_cast<long long>(blockIdx.x) * U / G;
-  const long long u_end = static_cast<long long>(blockIdx.x + 1) * U / G;
+  const long long u_begin = unit_start(a, blockIdx.x, G);
+  const long long u_end = unit_start(a, blockIdx.x + 1, G);
+  for (int c = threadIdx.x; c <= G; c += blockDim.x) starts[c] = static_cast<int>(unit_start(a, c, G));
   const long long limit = a.wait_limit;
   const int slots = static_cast<int>(a.stage_bytes / kBoxBytes);
 
@@ -359,8 +408,10 @@ __global__ void __launch_bounds__(kNormTcThreads, 1)
           }
         }
       }
-      mma_commit(drain);
-      mbar_wait(drain, 0, limit);
+      if (u_end > u_begin) {  // (an empty range issued no MMA to wait for)
+        mma_commit(drain);
+        mbar_wait(drain, 0, limit);
+      }
     }
   } else if (warp >= 6) {
     // ------------------------------------------------------- ||W_i||^2 warps
@@ -451,6 +502,15 @@ __global__ void __launch_bounds__(kNormTcThreads, 1)
       step();  // the W stages are the MMA thread's and the W^2 warps'
       if (!x.seg_last(a)) continue;
 
+      // segments of this M tile: the nonempty ranges meeting each of its chunks
+      // (counted while the segment's MMAs still run)
+      int expected = 0;
+      for (int c2 = 0; c2 < a.n_chunks; ++c2) {
+        const int s0 = (x.mt * a.n_chunks + c2) * a.kb_total;
+        const int o1 = unit_owner(starts, s0 + a.kb_total - 1, G);
+        for (int o = unit_owner(starts, s0, G); o <= o1; ++o) expected += unit_range_nonempty(starts, o) ? 1 : 0;
+      }
+
       // ---- segment epilogue: <B_i, V_i> over this chunk's columns
       if (!mbar_wait_warp(tmem_full, static_cast<uint32_t>(seg & 1), limit)) {
         if (lane == 0) record_timeout(a.status, abort_flag);
@@ -470,18 +530,15 @@ __global__ void __launch_bounds__(kNormTcThreads, 1)
         const int nb = min(slots, nbox - b0);
         for (int b = 0; b < nb; ++b) {
           const uint8_t* tile = sb + b * kBoxBytes;
+          const int j0 = (b0 + b) * kBK;
+          // the box's 64 columns of V in one TMEM round trip (the accumulator
+          // is allocated in a power of two of at least 64 columns)
+          float acc[64];
+          tmem_ld64(tmem_lane + j0, acc);
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int j0 = (b0 + b) * kBK + h * 32;
-            if (j0 >= x.n_this) break;
-            float acc[32];
-            tmem_ld32(tmem_lane + j0, acc);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              if (j0 + 8 * v < x.n_this)
-                dot += dot_bf16x8(*reinterpret_cast<const uint4*>(tile + sw128_chunk(row_local, h * 4 + v)),
-                                  acc + 8 * v);
-          }
+          for (int v = 0; v < 8; ++v)
+            if (j0 + 8 * v < x.n_this)
+              dot += dot_bf16x8(*reinterpret_cast<const uint4*>(tile + sw128_chunk(row_local, v)), acc + 8 * v);
         }
         release();
       }
@@ -501,7 +558,7 @@ __global__ void __launch_bounds__(kNormTcThreads, 1)
       if (lane == 0) mbar_arrive(w2_empty);
       const float partial = base_acc + a.two_s * dot;
       if (!deps_ready) {
-        grid_dep_wait();  // counters are zeroed by the Gram reduction kernel
+        grid_dep_wait();  // counters are zeroed by the Gram launch
         deps_ready = true;
       }
       a.partials[static_cast<size_t>(blockIdx.x + x.tc) * kBM + row_local] = partial;
@@ -509,11 +566,6 @@ __global__ void __launch_bounds__(kNormTcThreads, 1)
       // ---- the last of the M tile's segment-warps to arrive finishes the tile
       __threadfence();
       __syncwarp();
-      int expected = 0;
-      for (int c2 = 0; c2 < a.n_chunks; ++c2) {
-        const long long s0 = static_cast<long long>(x.mt * a.n_chunks + c2) * a.kb_total;
-        expected += stream_k_owner(s0 + a.kb_total - 1, U, G) - stream_k_owner(s0, U, G) + 1;
-      }
       int last = 0;
       if (lane == 0) last = (atomicAdd(&a.counters[x.mt], 1) == 4 * expected - 1);
       last = __shfl_sync(0xffffffffu, last, 0);
@@ -527,23 +579,25 @@ __global__ void __launch_bounds__(kNormTcThreads, 1)
         for (int j = 0; j < kRows; ++j) total[j] = 0.f;
         for (int c2 = 0; c2 < a.n_chunks; ++c2) {
           const int tc2 = x.mt * a.n_chunks + c2;
-          const long long s0 = static_cast<long long>(tc2) * a.kb_total;
-          const int o0 = stream_k_owner(s0, U, G);
-          const int o1 = stream_k_owner(s0 + a.kb_total - 1, U, G);
+          const int s0 = tc2 * a.kb_total;
+          const int o0 = unit_owner(starts, s0, G);
+          const int o1 = unit_owner(starts, s0 + a.kb_total - 1, G);
           for (int ob = o0; ob <= o1; ob += kFinOwners) {
             float v[kFinOwners][kRows];
+            bool use[kFinOwners];
+#pragma unroll
+            for (int k = 0; k < kFinOwners; ++k) use[k] = ob + k <= o1 && unit_range_nonempty(starts, ob + k);
 #pragma unroll
             for (int k = 0; k < kFinOwners; ++k)
 #pragma unroll
               for (int j = 0; j < kRows; ++j)
-                v[k][j] = (ob + k <= o1)
-                              ? ld_cg_f32(&a.partials[static_cast<size_t>(ob + k + tc2) * kBM + lane + 32 * j])
-                              : 0.f;
+                v[k][j] = use[k] ? ld_cg_f32(&a.partials[static_cast<size_t>(ob + k + tc2) * kBM + lane + 32 * j])
+                                 : 0.f;
 #pragma unroll
             for (int k = 0; k < kFinOwners; ++k)
 #pragma unroll
               for (int j = 0; j < kRows; ++j)
-                if (ob + k <= o1) total[j] += v[k][j];
+                if (use[k]) total[j] += v[k][j];
           }
         }
 #pragma unroll
@@ -582,8 +636,11 @@ __global__ void timeout_probe_kernel(long long limit, int* status) {
 // ===================================================================== Gram
 struct GramArgs {
   int r, kb_main, splits, n_tiles;
+  // 1: the first product is symmetric (A A^T) and only its tiles on or above
+  // the diagonal are computed, row-major over the upper triangle
+  int upper;
   long long wait_limit;
-  float* partial;  // [splits][n_tiles^2][128][128] fp32
+  float* partial;  // [splits][tiles][128][128] fp32; tiles = n_tiles^2, or n_tiles (n_tiles + 1) / 2 when upper
   int* status;
   // optional second product of the same r x r shape in the same launch:
   // CTAs from n_ctas1 on compute it from the second pair of maps
@@ -625,8 +682,21 @@ __global__ void __launch_bounds__(kNormThreads, 1)
   const CUtensorMap* const mapN = second ? &tmB2 : &tmB;
   const int split = bid % splits;
   const int tile = bid / splits;
-  const int mi = tile / a.n_tiles;
-  const int ni = tile % a.n_tiles;
+  const bool upper = a.upper && !second;
+  const int n_stored = upper ? a.n_tiles * (a.n_tiles + 1) / 2 : a.n_tiles * a.n_tiles;
+  int mi = tile / a.n_tiles;
+  int ni = tile % a.n_tiles;
+  if (upper) {
+    int t = tile;
+    mi = 0;
+    while (t >= a.n_tiles - mi) {
+      t -= a.n_tiles - mi;
+      ++mi;
+    }
+    ni = mi + t;
+  }
+  // a tile on the diagonal of A A^T has the same rows on both sides: one box per K block
+  const bool same = upper && mi == ni;
   const int n_this = min(kBoxRows, a.r - ni * kBoxRows);
   const int kb_lo = static_cast<int>(static_cast<long long>(split) * kb_main / splits);
   const int kb_hi = static_cast<int>(static_cast<long long>(split + 1) * kb_main / splits);
@@ -664,12 +734,12 @@ __global__ void __launch_bounds__(kNormThreads, 1)
       bool got = true;
       if (lane == 0) {
         got = mbar_wait(&empty[stage], phase ^ 1u, limit);
-        if (got) mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(2 * nk * kBoxBytes));
+        if (got) mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>((same ? 1 : 2) * nk * kBoxBytes));
         else record_timeout(a.status, abort_flag);
       }
       if (!__shfl_sync(0xffffffffu, got, 0)) break;
       __syncwarp();
-      if (lane < 2 * nk)
+      if (lane < 2 * nk && !(same && (lane & 1)))
         tma_load_2d(base_s + stage * kGramStageBytes + lane * kBoxBytes, (lane & 1) ? mapN : mapM, &full[stage],
                     (kb0 + (lane >> 1)) * kBK, ((lane & 1) ? ni : mi) * kBoxRows);
       parity_bits = (parity_bits & ~(1u << stage)) | (phase << stage);
@@ -698,8 +768,8 @@ __global__ void __launch_bounds__(kNormThreads, 1)
         for (int i = 0; i < nk; ++i)
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k)
-            mma_bf16(tmem, d0 + (2 * i) * (kBoxBytes >> 4) + 2 * k, d0 + (2 * i + 1) * (kBoxBytes >> 4) + 2 * k, idesc,
-                     (kb0 == kb_lo && i == 0 && k == 0) ? 0u : 1u);
+            mma_bf16(tmem, d0 + (2 * i) * (kBoxBytes >> 4) + 2 * k, d0 + (2 * i + (same ? 0 : 1)) * (kBoxBytes >> 4) + 2 * k,
+                     idesc, (kb0 == kb_lo && i == 0 && k == 0) ? 0u : 1u);
         mma_commit(&empty[stage]);
         if (++stage == kGramStages) {
           stage = 0;
@@ -715,7 +785,7 @@ __global__ void __launch_bounds__(kNormThreads, 1)
     const bool ok = mbar_wait_warp(tmem_full, 0, limit);
     if (ok && !__any_sync(0xffffffffu, *abort_flag != 0)) {
       tc_fence_after();
-      float* dst = partial + (static_cast<size_t>(split) * a.n_tiles * a.n_tiles + tile) * (kBoxRows * kBoxRows) +
+      float* dst = partial + (static_cast<size_t>(split) * n_stored + tile) * (kBoxRows * kBoxRows) +
                    static_cast<size_t>(row_local) * kBoxRows;
       for (int j0 = 0; j0 < n_this; j0 += 32) {
         float acc[32];
@@ -740,12 +810,18 @@ __global__ void __launch_bounds__(kNormThreads, 1)
 
 // Sums the K splits of G = A A^T in fixed order, scales by s/2 and writes the
 // bf16 G' the norm kernel's K extension reads; also zeroes the norm kernel's
-// tile counters.  CTAs from `g1` on reduce a second product the same way
+// tile counters.  With `upper`, the first product's partials hold only the
+// tiles on or above the diagonal, and an element below it is read from its
+// mirror.  CTAs from `g1` on reduce a second product the same way
 // (`partial2`, `splits2`, `scale2`, `Gs2`; a Gram launch of two products).
-__global__ void gram_reduce_kernel(const float* __restrict__ partial, int splits, int r, float half_s,
-                                   __nv_bfloat16* __restrict__ Gs, int* counters, int n_counters, int g1,
-                                   const float* __restrict__ partial2, int splits2, float scale2,
-                                   __nv_bfloat16* __restrict__ Gs2) {
+// 64 registers a thread at most (__launch_bounds__(256, 4)): a CTA of it then
+// fits beside a CTA of the norm kernel launched behind it, which can stream
+// W while the reduction still runs.
+__global__ void __launch_bounds__(256, 4)
+    gram_reduce_kernel(const float* __restrict__ partial, int splits, int r, float half_s,
+                       __nv_bfloat16* __restrict__ Gs, int* counters, int n_counters, int g1,
+                       const float* __restrict__ partial2, int splits2, float scale2,
+                       __nv_bfloat16* __restrict__ Gs2, int upper) {
   grid_dep_launch();
   grid_dep_wait();  // the Gram partial tiles are complete
   if (static_cast<int>(blockIdx.x) >= g1) {
@@ -754,15 +830,17 @@ __global__ void gram_reduce_kernel(const float* __restrict__ partial, int splits
     half_s = scale2;
     Gs = Gs2;
     n_counters = 0;
+    upper = 0;
   }
   const int bx = static_cast<int>(blockIdx.x) >= g1 ? static_cast<int>(blockIdx.x) - g1 : static_cast<int>(blockIdx.x);
   const int gx = static_cast<int>(blockIdx.x) >= g1 ? static_cast<int>(gridDim.x) - g1 : g1;
   const long long total = static_cast<long long>(r) * r;
   const int nt = (r + kBoxRows - 1) / kBoxRows;
-  const long long split_stride = static_cast<long long>(nt) * nt * kBoxRows * kBoxRows;
-  // four elements per thread and eight splits per round: 32 independent loads
+  const long long split_stride =
+      static_cast<long long>(upper ? nt * (nt + 1) / 2 : nt * nt) * kBoxRows * kBoxRows;
+  // four elements per thread and four splits per round: 16 independent loads
   // in flight; each element still adds its splits in increasing order
-  constexpr int kE = 4, kS = 8;
+  constexpr int kE = 4, kS = 4;
   const long long step = static_cast<long long>(gx) * blockDim.x;
   for (long long base = bx * static_cast<long long>(blockDim.x) + threadIdx.x; base < total;
        base += kE * step) {
@@ -771,10 +849,24 @@ __global__ void gram_reduce_kernel(const float* __restrict__ partial, int splits
 #pragma unroll
     for (int e = 0; e < kE; ++e) {
       const long long idx = min(base + e * step, total - 1);
-      const int j = static_cast<int>(idx / r);
-      const int k = static_cast<int>(idx - static_cast<long long>(j) * r);
-      src[e] = (static_cast<long long>(j / kBoxRows) * nt + k / kBoxRows) * kBoxRows * kBoxRows +
-               static_cast<long long>(j % kBoxRows) * kBoxRows + (k % kBoxRows);
+      int j = static_cast<int>(idx / r);
+      int k = static_cast<int>(idx - static_cast<long long>(j) * r);
+      int ti = j / kBoxRows, tk = k / kBoxRows;
+      long long tile;
+      if (upper) {
+        if (ti > tk) {  // below the diagonal: G[j][k] = G[k][j]
+          const int t = j;
+          j = k;
+          k = t;
+          const int tt = ti;
+          ti = tk;
+          tk = tt;
+        }
+        tile = static_cast<long long>(ti) * nt - static_cast<long long>(ti) * (ti - 1) / 2 + (tk - ti);
+      } else {
+        tile = static_cast<long long>(ti) * nt + tk;
+      }
+      src[e] = tile * kBoxRows * kBoxRows + static_cast<long long>(j % kBoxRows) * kBoxRows + (k % kBoxRows);
       sum[e] = 0.f;
     }
     for (int s0 = 0; s0 < splits; s0 += kS) {

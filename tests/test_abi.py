@@ -189,30 +189,80 @@ def test_num_sms_without_device(lib):
 
 
 # ------------------------------------------------ stream-K schedule algebra
-def _owner(u, U, G):
-    return ((u + 1) * G - 1) // U
+# A mirror of the norm kernel's schedule: weighted contiguous unit ranges,
+# the owner search over them, and the rotated walk of one range.
+def _cum(c, early, w_e, w_l):
+    return w_e * min(c, early) + w_l * max(0, c - early)
 
 
-@pytest.mark.parametrize("U,G", [(1, 1), (3, 3), (7, 3), (8384, 148), (134 * 216, 148), (10, 7)])
-def test_stream_k_partition(U, G):
-    """Ranges [floor(cU/G), floor((c+1)U/G)) tile [0, U); owner() inverts them;
-    segment index c + tc is unique when segments split at tile boundaries."""
-    ranges = [(c * U // G, (c + 1) * U // G) for c in range(G)]
+def _start(c, U, G, early, w_e, w_l):
+    return U * _cum(c, early, w_e, w_l) // _cum(G, early, w_e, w_l)
+
+
+def _owner(u, U, G, early, w_e, w_l):
+    lo, hi = 0, G - 1
+    while lo < hi:
+        mid = (lo + hi + 1) // 2
+        if _start(mid, U, G, early, w_e, w_l) <= u:
+            lo = mid
+        else:
+            hi = mid - 1
+    return lo
+
+
+def _walk(u0, u1, kb_total):
+    """Units of [u0, u1) in walk order with the segment-end flags: from the
+    first tile boundary tb on, then [u0, tb)."""
+    tb = min(u1, -(-u0 // kb_total) * kb_total)
+    order = list(range(tb, u1)) + list(range(u0, tb)) if u0 < tb < u1 else list(range(u0, u1))
+    len2 = tb - u0 if u0 < tb < u1 else 0
+    out = []
+    for i, u in enumerate(order):
+        left = len(order) - i
+        last = left == 1 or u % kb_total == kb_total - 1 or (len2 > 0 and left == len2 + 1)
+        out.append((u, last))
+    return out
+
+
+@pytest.mark.parametrize("U,G,early,w_e,w_l", [(1, 1, 1, 1, 1), (3, 3, 3, 1, 1), (7, 3, 3, 5, 5), (8384, 148, 148, 16, 16),
+                                               (134 * 216, 148, 124, 3139, 2900), (10, 7, 5, 16, 0), (8576, 148, 124, 945, 730),
+                                               (300, 148, 140, 40, 2)])
+def test_stream_k_partition(U, G, early, w_e, w_l):
+    """Weighted ranges tile [0, U); the owner search inverts them; the rotated
+    walk visits each unit once, in segments of one tile each; a tile's
+    segments are the nonempty ranges meeting it; segment slot c + tile is
+    unique."""
+    ranges = [(_start(c, U, G, early, w_e, w_l), _start(c + 1, U, G, early, w_e, w_l)) for c in range(G)]
     assert ranges[0][0] == 0 and ranges[-1][1] == U
     for (a0, a1), (b0, b1) in zip(ranges, ranges[1:]):
-        assert a1 == b0
+        assert a1 == b0 and a0 <= a1
     for c, (a, b) in enumerate(ranges):
         for u in range(a, b):
-            assert _owner(u, U, G) == c
+            assert _owner(u, U, G, early, w_e, w_l) == c
     for kb_total in (1, 3, 134):
         seen = set()
+        segs = {}
         for c, (a, b) in enumerate(ranges):
-            for u in range(a, b):
-                if u == a or u % kb_total == 0:
-                    idx = c + u // kb_total
+            walk = _walk(a, b, kb_total)
+            assert sorted(u for u, _ in walk) == list(range(a, b))
+            seg = []
+            for u, last in walk:
+                seg.append(u)
+                if last:
+                    tiles = {v // kb_total for v in seg}
+                    assert len(tiles) == 1 and seg == list(range(seg[0], seg[-1] + 1))
+                    t = tiles.pop()
+                    segs[t] = segs.get(t, 0) + 1
+                    idx = c + t
                     assert idx not in seen
                     seen.add(idx)
+                    seg = []
+            assert not seg
         assert max(seen, default=0) < G + (U + kb_total - 1) // kb_total
+        for t, n in segs.items():
+            o0 = _owner(t * kb_total, U, G, early, w_e, w_l)
+            o1 = _owner(min(U, (t + 1) * kb_total) - 1, U, G, early, w_e, w_l)
+            assert n == sum(1 for o in range(o0, o1 + 1) if ranges[o][1] > ranges[o][0])
 
 
 def test_fused_linear_argument_errors(lib):
