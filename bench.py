@@ -75,7 +75,7 @@ def load_peaks():
 
 # the sources that define each measured kernel family's code and launches
 TRAFFIC_SOURCES = {
-    "norm": ("sm100_ptx.cuh", "norm_tc.cuh", "dora_api.cu"),
+    "norm": ("sm100_ptx.cuh", "norm_tc.cuh", "gram_cluster.cuh", "dora_api.cu"),
     "compose_fwd": ("sm100_ptx.cuh", "compose.cuh", "dora_api.cu"),
     "compose_bwd": ("sm100_ptx.cuh", "compose.cuh", "dora_api.cu"),
 }
@@ -94,8 +94,9 @@ def source_digest(names=None):
 
 
 def load_traffic():
-    """DRAM bytes per launch from the committed ncu summary, valid only for the
-    kernel sources it was captured from."""
+    """DRAM bytes per launch from the committed ncu summary, keyed by (kernel,
+    workload label): valid only for the workload it was captured on and for
+    the kernel sources it was captured from."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     out = {}
     if not os.path.exists(p):
@@ -104,8 +105,33 @@ def load_traffic():
         parts = line.split()
         if len(parts) >= 4 and not line.startswith("#") and parts[0] in TRAFFIC_SOURCES:
             if parts[1] == source_digest(TRAFFIC_SOURCES[parts[0]]):
-                out[parts[0]] = {"bytes": float(parts[2]), "workload": parts[3]}
+                out[(parts[0], parts[3])] = float(parts[2])
     return out
+
+
+def traffic_labels(wl):
+    """Workload labels of the traffic rows: the norm's depends on the weights'
+    shape, the compose kernels' on the token count too."""
+    return {"norm": wl.name, "compose_fwd": f"{wl.name}_T{wl.tokens}", "compose_bwd": f"{wl.name}_T{wl.tokens}"}
+
+
+L2_BYTES = 126 << 20
+
+
+def step_bytes(wl):
+    e = 2 if wl.dtype == "bf16" else 4
+    return norm_bytes(wl.d_out, wl.d_in, wl.r, e) + fwd_bytes(wl.tokens, wl.d_out, e) + bwd_bytes(wl.tokens, wl.d_out, e)
+
+
+def l2_statement(wl, flushed):
+    mb = step_bytes(wl) / 1e6
+    if flushed:
+        return (f"flushed before every step (256 MB written, then 256 MB read; untimed): a step streams only "
+                f"{mb:.0f} MB against a 126 MB L2")
+    return f"no flush: each step streams {mb:.0f} MB (norm inputs, then 3 activation reads + 1 write, then 3 reads + 2 writes)"
+
+
+DTYPE_LABEL = {"bf16": "bf16", "f32": "f32"}
 
 
 # ---------------------------------------------------------------- clocks
@@ -188,8 +214,12 @@ def run_ours(args, rank, world, local_rank):
     ws_n = torch.empty(D.dora_factored_norm_workspace_size(d_out, d_in, r), dtype=torch.uint8, device=dev)
     ws_b = torch.empty(D.dora_compose_bwd_workspace_size(T, d_out), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    # a workload whose step fits in L2 twice over is flushed before every step
+    flush = L2Flush(dev) if step_bytes(wl) < 2 * L2_BYTES else None
 
     def step(ev=None):
+        if flush is not None:
+            flush()
         if ev is not None:
             ev[0].record(stream)
         D.dora_factored_norm(W, A, B, s, n_out=n, workspace=ws_n)
@@ -215,8 +245,10 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
+    launches0 = D.dora_launch_count()
     for k in range(args.steps):
         step(evs[k])
+    launches = D.dora_launch_count() - launches0
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
@@ -227,6 +259,8 @@ def run_ours(args, rank, world, local_rank):
     t_fwd = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps * 1e-3
     t_bwd = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps * 1e-3
     t_total = evs[0][0].elapsed_time(evs[-1][3]) * 1e-3
+    if flush is not None:  # the flushes between steps are not the step's
+        t_total = (t_norm + t_fwd + t_bwd) * args.steps
     t_total, t_norm, t_fwd, t_bwd = max_over_ranks([t_total, t_norm, t_fwd, t_bwd], world, dev)
 
     # ---- end to end through the Python API with pinned host buffers
@@ -245,7 +279,8 @@ def run_ours(args, rank, world, local_rank):
     norm_bwd = idle_then(lambda: run_norm_backward_context(D, dev, wl, W, A, B, n)) if bf16_ctx else None
     fused = idle_then(lambda: run_fused_linear_context(D, dev, wl, W, A, B, m, n)) if bf16_ctx else None
     return dict(t_total=t_total, t_norm=t_norm, t_fwd=t_fwd, t_bwd=t_bwd, clocks=clocks, status=status, e2e=e2e,
-                wl=wl, dense=dense, batched=batched, fused=fused, norm_bwd=norm_bwd)
+                wl=wl, dense=dense, batched=batched, fused=fused, norm_bwd=norm_bwd, launches=launches,
+                flushed=flush is not None)
 
 
 def run_dense_comparator(D, dev, W, A, B, s, ws_n, reps=10):
@@ -561,10 +596,12 @@ def build_line(args, res, N, peaks, peak_src, traffic, cpu):
     """The JSON line of our arm from the max-over-ranks times in `res`; N ranks
     each ran one replica of the workload, so every rate is the whole job's."""
     wl = res["wl"]
+    e = 2 if wl.dtype == "bf16" else 4
     F = norm_flops(wl.d_out, wl.d_in, wl.r)
-    Bn = norm_bytes(wl.d_out, wl.d_in, wl.r)
-    Bf = fwd_bytes(wl.tokens, wl.d_out)
-    Bb = bwd_bytes(wl.tokens, wl.d_out)
+    Bn = norm_bytes(wl.d_out, wl.d_in, wl.r, e)
+    Bf = fwd_bytes(wl.tokens, wl.d_out, e)
+    Bb = bwd_bytes(wl.tokens, wl.d_out, e)
+    labels = traffic_labels(wl)
 
     def roof(kernel, t, work, bound):
         if bound == "tensor":
@@ -575,10 +612,9 @@ def build_line(args, res, N, peaks, peak_src, traffic, cpu):
             ach = work / t / 1e9
             pk = peaks["hbm_gbs"]
             unit = "GB/s"
-        tr = traffic.get(kernel)
         return {"kernel": kernel, "bound": bound, "achieved": ach, "peak": pk, "unit": unit, "frac": ach / pk,
-                "traffic": tr["bytes"] if tr else None, "peak_source": f"{peak_src} (burst)" if bound == "tensor" else peak_src,
-                "time_us": t * 1e6}
+                "traffic": traffic.get((kernel, labels[kernel])),
+                "peak_source": f"{peak_src} (burst)" if bound == "tensor" else peak_src, "time_us": t * 1e6}
 
     # norm bound: slower of FLOPs at tensor peak and bytes at HBM bandwidth
     norm_bound = "tensor" if F / (peaks["bf16_tflops"] * 1e12) >= Bn / (peaks["hbm_gbs"] * 1e9) else "hbm"
@@ -591,7 +627,6 @@ def build_line(args, res, N, peaks, peak_src, traffic, cpu):
     e2e = res["e2e"]
     e2e_norm = F * N / (e2e["t_norm"]) / 1e12
 
-    launches_per_step = 3 + 1 + 1  # gram, gram_reduce, norm; compose fwd; compose bwd
     line = {
         "metric": METRIC,
         "value": F * N / res["t_norm"] / 1e12,
@@ -603,11 +638,10 @@ def build_line(args, res, N, peaks, peak_src, traffic, cpu):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": DTYPE_LABEL[wl.dtype],
         "data": "synthetic",
         "config": {"workload": wl.name, "d_out": wl.d_out, "d_in": wl.d_in, "r": wl.r, "tokens": wl.tokens,
-                   "s": wl.s, "parallelism": f"replicas x{N}",
-                   "l2": "no flush: each step streams > 1 GB (W 134 MB, 3 activation reads + 3 writes of 134 MB)"},
+                   "s": wl.s, "parallelism": f"replicas x{N}", "l2": l2_statement(wl, res["flushed"])},
         "value_basis": "norm FLOPs x ranks / max-over-ranks mean CUDA-event time of the norm launches in the timed steps",
         "compose": {
             "fwd": {"value": Bf * N / res["t_fwd"] / 1e9, "unit": "GB/s", "frac": rl[1]["frac"],
@@ -628,7 +662,8 @@ def build_line(args, res, N, peaks, peak_src, traffic, cpu):
                 "basis": "norm FLOPs / (H2D of W, A, B + norm + D2H of n), pinned host buffers",
                 "compose_fwd_gbs": Bf * N / e2e["t_fwd"] / 1e9, "compose_bwd_gbs": Bb * N / e2e["t_bwd"] / 1e9},
         "cpu_baseline": cpu,
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": res["launches"],
+        "gpu_launches_basis": "dora_launch_count() after the timed steps minus before them (this rank)",
         "memset_nodes": 0,  # the compose backward's counters are tagged per call, nothing is cleared
         "clocks": res["clocks"],
         "device_status": res["status"],
@@ -707,13 +742,24 @@ def run_sweep(args):
 
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    stream = torch.cuda.current_stream(dev)
     peaks, peak_src = load_peaks()
     reps = max(5, min(args.steps, 50))
-    flush = L2Flush(dev)
-    pts = []
     sampler = ClockSampler(0)
     sampler.start()
+    pts = sweep_points(D, dev, reps, peaks)
+    clocks = sampler.stop()
+    status = D.dora_device_status()
+    print(json.dumps({"sweep": pts, "reps_per_point": reps, "l2": "before every timed call 256 MB written, then another 256 MB read",
+                      "peaks": {"bf16_tflops": peaks["bf16_tflops"], "hbm_gbs": peaks["hbm_gbs"],
+                                "source": peak_src}, "clocks": clocks, "device_status": status}), flush=True)
+    return 0 if status == D.DORA_OK else 1
+
+
+def sweep_points(D, dev, reps, peaks):
+    """Points of the rank/shape sweep (see run_sweep)."""
+    stream = torch.cuda.current_stream(dev)
+    flush = L2Flush(dev)
+    pts = []
     for wl in WL.RANK_SWEEP:
         W, A, B, _ = WL.make_weights(wl, dev)
         n = torch.empty(wl.d_out, dtype=torch.float32, device=dev)
@@ -744,12 +790,142 @@ def run_sweep(args):
             pts.append({"op": op, "tokens": wl.tokens, "d_out": wl.d_out, "us": t * 1e6, "gbs": by / t * 1e-9,
                         "bound": "hbm", "roofline_frac": by / t * 1e-9 / peaks["hbm_gbs"]})
         del base, lora, dy, y, d_base, d_lora, ws
-    clocks = sampler.stop()
-    status = D.dora_device_status()
-    print(json.dumps({"sweep": pts, "reps_per_point": reps, "l2": "before every timed call 256 MB written, then another 256 MB read",
-                      "peaks": {"bf16_tflops": peaks["bf16_tflops"], "hbm_gbs": peaks["hbm_gbs"],
-                                "source": peak_src}, "clocks": clocks, "device_status": status}), flush=True)
-    return 0 if status == D.DORA_OK else 1
+    return pts
+
+
+# --------------------------------------------------- the other configs
+def kernel_point(kernel, t, flops, nbytes, peaks, traffic, label):
+    """One kernel's time against its roofline time: the slower of its FLOPs
+    at the measured bf16 peak and its bytes at the measured copy bandwidth."""
+    t_tensor = flops / (peaks["bf16_tflops"] * 1e12) if flops else 0.0
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    bound = "tensor" if t_tensor >= t_hbm else "hbm"
+    pt = {"kernel": kernel, "time_us": t * 1e6, "bound": bound, "roofline_time_us": max(t_tensor, t_hbm) * 1e6,
+          "frac": max(t_tensor, t_hbm) / t, "gbs": nbytes / t / 1e9,
+          "traffic": traffic.get((kernel, label))}
+    if flops:
+        pt["tflops"] = flops / t / 1e12
+    return pt
+
+
+def config_line(D, dev, wl, what, peaks, traffic, reps, full_step=False):
+    """Norm, compose forward and compose backward of workload `wl`, each timed
+    alone after an L2 flush (median of `reps` calls); with `full_step`, also
+    the three back to back, as one training step of the adapter path."""
+    stream = torch.cuda.current_stream(dev)
+    flush = L2Flush(dev)
+    e = 2 if wl.dtype == "bf16" else 4
+    W, A, B, _ = WL.make_weights(wl, dev)
+    m, n_ref = WL.make_near_unity_mn(wl, W, dev)
+    _, base, lora = WL.make_activations(wl, W, A, B, dev)
+    dy = WL.make_grad(wl, dev)
+    n = torch.empty(wl.d_out, dtype=torch.float32, device=dev)
+    y, d_base, d_lora = torch.empty_like(base), torch.empty_like(base), torch.empty_like(base)
+    d_m = torch.empty(wl.d_out, dtype=torch.float32, device=dev)
+    ws_n = torch.empty(D.dora_factored_norm_workspace_size(wl.d_out, wl.d_in, wl.r, WL.torch_dtype(wl)),
+                       dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(D.dora_compose_bwd_workspace_size(wl.tokens, wl.d_out), dtype=torch.uint8, device=dev)
+    norm = lambda: D.dora_factored_norm(W, A, B, wl.s, n_out=n, workspace=ws_n)  # noqa: E731
+    fwd = lambda: D.dora_compose_fwd(base, lora, m, n_ref, wl.s, y=y)  # noqa: E731
+    bwd = lambda: D.dora_compose_bwd(dy, base, lora, m, n_ref, wl.s, d_base, d_lora, d_m, ws_b)  # noqa: E731
+    launches0 = D.dora_launch_count()
+    t_n = time_alone(norm, reps, flush, stream)
+    t_f = time_alone(fwd, reps, flush, stream)
+    t_b = time_alone(bwd, reps, flush, stream)
+    labels = traffic_labels(wl)
+    line = {
+        "config_line": what, "workload": wl.name, "dtype": DTYPE_LABEL[wl.dtype],
+        "config": {"d_out": wl.d_out, "d_in": wl.d_in, "r": wl.r, "tokens": wl.tokens, "s": wl.s},
+        "l2": "every call timed alone after 256 MB written, then another 256 MB read (untimed)",
+        "reps_per_kernel": reps,
+        "kernels": [
+            kernel_point("norm", t_n, norm_flops(wl.d_out, wl.d_in, wl.r), norm_bytes(wl.d_out, wl.d_in, wl.r, e),
+                         peaks, traffic, labels["norm"]),
+            kernel_point("compose_fwd", t_f, 0, fwd_bytes(wl.tokens, wl.d_out, e), peaks, traffic, labels["compose_fwd"]),
+            kernel_point("compose_bwd", t_b, 0, bwd_bytes(wl.tokens, wl.d_out, e), peaks, traffic, labels["compose_bwd"]),
+        ],
+    }
+    if full_step:
+        def step():
+            norm()
+            fwd()
+            bwd()
+        t_s = time_alone(step, reps, flush, stream)
+        roof = sum(k["roofline_time_us"] for k in line["kernels"])
+        line["full_step"] = {"time_us": t_s * 1e6, "roofline_time_us": roof, "frac": roof / (t_s * 1e6),
+                             "what": "norm -> compose fwd -> compose bwd back to back after one flush"}
+    line["gpu_launches"] = D.dora_launch_count() - launches0
+    line["device_status"] = D.dora_device_status()
+    return line
+
+
+def oracle_single_thread_line(wl):
+    """The oracle on the whole tiny workload with its BLAS limited to one
+    thread: norm, compose forward, compose backward (median of 20 runs)."""
+    import numpy as np
+
+    import oracle
+
+    try:
+        from threadpoolctl import threadpool_limits
+    except Exception:  # pragma: no cover - threadpoolctl is in the image
+        threadpool_limits = None
+    W, A, B, m = WL.make_weights(wl)
+    W64, A64, B64 = (t.double().numpy() for t in (W, A, B))
+    rng = np.random.default_rng(0)
+    base = rng.standard_normal((wl.tokens, wl.d_out))
+    lora = rng.standard_normal((wl.tokens, wl.d_out)) * 0.02
+    dy = rng.standard_normal((wl.tokens, wl.d_out))
+    mm = m.double().numpy()
+
+    def timed(f):
+        ts = []
+        for _ in range(20):
+            t0 = time.perf_counter()
+            f()
+            ts.append(time.perf_counter() - t0)
+        return statistics.median(ts)
+
+    def run():
+        n = oracle.row_norm(W64, A64, B64, wl.s)
+        return (timed(lambda: oracle.row_norm(W64, A64, B64, wl.s)),
+                timed(lambda: oracle.compose_forward(base, lora, mm, n, wl.s)),
+                timed(lambda: oracle.compose_backward(dy, base, lora, mm, n, wl.s)))
+
+    if threadpool_limits is not None:
+        with threadpool_limits(limits=1):
+            t_n, t_f, t_b = run()
+    else:
+        t_n, t_f, t_b = run()
+    return {"config_line": "config-1 oracle, one thread", "workload": wl.name, "kind": "oracle", "cores": 1,
+            "config": {"d_out": wl.d_out, "d_in": wl.d_in, "r": wl.r, "tokens": wl.tokens, "s": wl.s},
+            "norm_us": t_n * 1e6, "compose_fwd_us": t_f * 1e6, "compose_bwd_us": t_b * 1e6,
+            "norm_tflops": norm_flops(wl.d_out, wl.d_in, wl.r) / t_n / 1e12,
+            "sample": "the whole workload, median of 20 runs each"}
+
+
+def run_config_lines(args, peaks):
+    """The other configs on this GPU, one JSON line each, after the headline line."""
+    from factored_weight_norm_b200 import dora as D
+
+    dev = torch.device("cuda", 0)
+    traffic = load_traffic()
+    reps = max(5, min(args.steps, 20))
+    lines = [
+        config_line(D, dev, WL.TINY_F32, "config-1 tiny fp32", peaks, traffic, reps),
+        config_line(D, dev, WL.SINGLE_4096, "config-2 bf16 single module", peaks, traffic, reps),
+        config_line(D, dev, WL.MLP_UP_32B, "config-4 bf16 MLP up-projection, training step", peaks, traffic, reps,
+                    full_step=True),
+    ]
+    sampler = ClockSampler(0)
+    sampler.start()
+    pts = sweep_points(D, dev, reps, peaks)
+    lines.append({"config_line": "config-5 rank/token sweep", "sweep": pts, "reps_per_point": reps,
+                  "l2": "every call timed alone after 256 MB written, then another 256 MB read (untimed)",
+                  "clocks": sampler.stop(), "device_status": D.dora_device_status()})
+    if not args.no_cpu_baseline:
+        lines.append(oracle_single_thread_line(WL.TINY_F32))
+    return lines
 
 
 # ------------------------------------------------------------------- main
@@ -766,6 +942,9 @@ def main():
     ap.add_argument("--no-context", action="store_true",
                     help="skip the context measurements after the timed step (dense comparator, many modules, "
                          "fused linear, attached-norm backward), e.g. for a profiler's launch list")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the lines of the other configs (tiny fp32, 4096 single module, MLP up-projection "
+                         "step, rank/token sweep, single-thread oracle) after the headline line")
     ap.add_argument("--sweep", action="store_true",
                     help="run the rank/shape sweep (norm over ranks, compose over token counts) on one GPU "
                          "and print its points instead of the benchmark line")
@@ -807,6 +986,9 @@ def main():
 
     if rank == 0:
         print(json.dumps(build_line(args, res, N, peaks, peak_src, traffic, cpu)), flush=True)
+    if rank == 0 and N == 1 and not args.no_configs and wl.name == WL.HEADLINE.name and args.tokens is None:
+        for line in run_config_lines(args, peaks):
+            print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
     return 0

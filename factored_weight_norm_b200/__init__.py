@@ -22,6 +22,7 @@ from .dora import (  # noqa: F401
     dora_factored_norm_workspace_size,
     dora_fused_linear_fwd,
     dora_fused_linear_fwd_workspace_size,
+    dora_launch_count,
     dora_norm_finish,
     dora_num_sms,
     dora_status_string,

@@ -68,7 +68,7 @@ int pair_attrs(K kernel, int smem_optin) {
 }
 constexpr int kMaxGrid = 1024;                         // bound on the persistent grid
 constexpr int kMaxGramSplits = 32;
-constexpr int kGramBlocksPerSplit = 32;                // K blocks a Gram CTA of the norm takes, about
+constexpr int kGramMinBlocks = 4;                      // fewest K blocks a Gram CTA of the norm takes
 constexpr int kMaxBwdChunks = 64;
 constexpr int kMaxDevices = 64;
 constexpr int64_t kMaxRank = 4096;
@@ -85,6 +85,11 @@ struct DeviceInfo {
 };
 
 std::mutex g_mu;
+
+// Kernels this library has launched in this process (every launch site
+// counts itself once, before it launches).
+std::atomic<unsigned long long> g_launches{0};
+inline void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 DeviceInfo g_dev[kMaxDevices];
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -203,6 +208,7 @@ void launch_compose_bwd(dim3 grid, cudaStream_t st, const void* dy, const void* 
                         long long d_out, void* d_base, void* d_lora, float* part, unsigned long long* cnt, float* d_m,
                         long long rows) {
   auto kernel = bias ? compose_bwd_kernel<T, VEC, true> : compose_bwd_kernel<T, VEC, false>;
+  note_launch();
   kernel<<<grid, kBwdThreads, 0, st>>>(static_cast<const T*>(dy), static_cast<const T*>(base_out),
                                        static_cast<const T*>(lora_out), static_cast<const T*>(bias), m, n, s, tokens,
                                        nvec, d_out, static_cast<T*>(d_base), static_cast<T*>(d_lora), part, cnt, d_m,
@@ -289,11 +295,12 @@ int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_
   // for the Gram launch only there.
   const int nt = static_cast<int>(cdiv(r, kBoxRows));
   const int up_tiles = nt * (nt + 1) / 2;
-  // about kGramBlocksPerSplit K blocks per CTA, on at most a third of the
-  // SMs; a power of two up to 8 (the cluster size)
+  // as many K splits as a cluster holds (8), while each keeps at least
+  // kGramMinBlocks K blocks and the clusters take at most a third of the
+  // SMs: the Gram latency then stays well inside the GEMM's, small
+  // problems included
   int splits = 1;
-  while (splits < 8 && splits * kGramBlocksPerSplit < p.kb_main && 2 * splits <= p.kb_main &&
-         up_tiles * 2 * splits <= std::max(1, dev->num_sms / 3))
+  while (splits < 8 && 2 * splits * kGramMinBlocks <= p.kb_main && up_tiles * 2 * splits <= std::max(1, dev->num_sms / 3))
     splits *= 2;
   {
     GramClusterArgs gca{};
@@ -319,6 +326,7 @@ int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_
     gcfg.blockDim = dim3(kGcThreads);
     gcfg.dynamicSmemBytes = kGcSmem;
     cudaError_t e = cudaSuccess;
+    note_launch();
     switch (splits) {
       case 1: e = cudaLaunchKernelEx(&gcfg, gram_cluster_kernel<1>, tmA, gca); break;
       case 2: e = cudaLaunchKernelEx(&gcfg, gram_cluster_kernel<2>, tmA, gca); break;
@@ -384,6 +392,7 @@ int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kNormTcThreads);
   cfg.dynamicSmemBytes = static_cast<size_t>(na.stages) * (na.stage_bytes + 16) + smem_fixed;
+  note_launch();
   if (cudaLaunchKernelEx(&cfg, norm_tc_kernel, tmW, tmA, tmB, tmG, na) != cudaSuccess) return DORA_ERR_CUDA;
   return launch_error();
 }
@@ -490,6 +499,7 @@ int norm_batched(const dora_norm_problem* q, const BatchLayout& L, uint8_t* ws, 
 
   const BatchDesc* d_descs = reinterpret_cast<const BatchDesc*>(ws);
   const size_t gram_smem = kGramStages * kGramStageBytes + (2 * kGramStages + 1) * 8 + 16 + 1024;
+  note_launch();
   gram_batched_kernel<<<ng, kNormThreads, gram_smem, st>>>(d_descs, reinterpret_cast<const BatchItem*>(ws + L.off_gitems),
                                                           kWaitLimitCycles, dev->status);
   if (launch_error()) return DORA_ERR_CUDA;
@@ -512,6 +522,7 @@ int norm_batched(const dora_norm_problem* q, const BatchLayout& L, uint8_t* ws, 
   cfg.gridDim = dim3(static_cast<unsigned>(std::min<long long>({static_cast<long long>(dev->num_sms), ni, kMaxGrid})));
   cfg.blockDim = dim3(kNormThreads);
   cfg.dynamicSmemBytes = static_cast<size_t>(a.stages) * a.stage_bytes + (2 * a.stages + 3) * 8 + 16 + 1024;
+  note_launch();
   if (cudaLaunchKernelEx(&cfg, norm_batched_kernel, d_descs, reinterpret_cast<const BatchItem*>(ws + L.off_items), a) !=
       cudaSuccess)
     return DORA_ERR_CUDA;
@@ -571,6 +582,7 @@ int dora_norm_finish(float* n, int64_t d_out, void* stream) {
   if (!aligned(n, 4)) return DORA_ERR_UNSUPPORTED;
   DeviceInfo* dev = nullptr;
   if (device_info(&dev)) return DORA_ERR_CUDA;
+  note_launch();
   norm_finish_kernel<<<static_cast<unsigned>(cdiv(d_out, 256)), 256, 0, static_cast<cudaStream_t>(stream)>>>(n, d_out);
   return launch_error();
 }
@@ -595,6 +607,7 @@ int factored_norm(const void* W, const void* A, const void* B, int64_t d_out, in
   }
   if (r == 0) {
     const int blocks = static_cast<int>(cdiv(d_out, 8));
+    note_launch();
     if (dt == DORA_BF16)
       rownorm_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(W), static_cast<int>(d_out),
                                                             static_cast<int>(d_in), n_out, squared ? 1 : 0);
@@ -607,8 +620,10 @@ int factored_norm(const void* W, const void* A, const void* B, int64_t d_out, in
   float* G = static_cast<float*>(workspace);
   const long long pairs = r * (r + 1) / 2;
   const int gblocks = static_cast<int>(std::min<long long>(cdiv(pairs, 8), 8LL * dev->num_sms));
+  note_launch();
   gram_f32_kernel<<<gblocks, 256, 0, st>>>(static_cast<const float*>(A), static_cast<int>(r), static_cast<int>(d_in), G);
   if (launch_error()) return DORA_ERR_CUDA;
+  note_launch();
   norm_f32_kernel<<<static_cast<unsigned>(d_out), 256, 0, st>>>(
       static_cast<const float*>(W), static_cast<const float*>(A), static_cast<const float*>(B), G,
       static_cast<int>(d_out), static_cast<int>(d_in), static_cast<int>(r), s, n_out, squared ? 1 : 0);
@@ -655,6 +670,7 @@ int dora_compose_fwd_bias(const void* base_out, const void* lora_out, const void
   const long long rows = cdiv(tokens, gy);
   const long long gy2 = cdiv(tokens, rows);
   dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy2));
+  note_launch();
   if (dt == DORA_BF16)
     compose_fwd_kernel<__nv_bfloat16, 8><<<grid, threads, 0, st>>>(
         static_cast<const __nv_bfloat16*>(base_out), static_cast<const __nv_bfloat16*>(lora_out),
@@ -803,9 +819,12 @@ int dora_selftest_timeout(int64_t limit_cycles, void* stream) {
   if (limit_cycles <= 0 || limit_cycles > kWaitLimitCycles) return DORA_ERR_INVALID_ARG;
   DeviceInfo* dev = nullptr;
   if (device_info(&dev)) return DORA_ERR_CUDA;
+  note_launch();
   timeout_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_cycles, dev->status);
   return launch_error();
 }
+
+uint64_t dora_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int dora_num_sms(void) {
   int n = 0;
@@ -892,6 +911,7 @@ int dora_fused_linear_fwd(const void* x, const void* W, const void* A, const voi
     pa.status = dev->status;
     cfg.numAttrs = 1;  // cluster shape only: ordered after everything before it on the stream
     cfg.gridDim = dim3(pairs_for(static_cast<long long>(pa.tiles_m) * pa.tiles_n));
+    note_launch();
     if (cudaLaunchKernelEx(&cfg, linear_pair_kernel<false, false>, tmX, tmA, tmX, tmA, pa) != cudaSuccess)
       return DORA_ERR_CUDA;
   }
@@ -919,6 +939,7 @@ int dora_fused_linear_fwd(const void* x, const void* W, const void* A, const voi
   cfg.gridDim = dim3(pairs_for(static_cast<long long>(la.tiles_m) * la.tiles_n));
   const CUtensorMap& tmA2 = r > 0 ? tmP : tmX;
   const CUtensorMap& tmB2 = r > 0 ? tmB : tmW;
+  note_launch();
   if (cudaLaunchKernelEx(&cfg, linear_pair_kernel<false, false>, tmX, tmW, tmA2, tmB2, la) != cudaSuccess)
     return DORA_ERR_CUDA;
   return launch_error();
@@ -1002,6 +1023,7 @@ int dora_factored_norm_bwd(const void* W, const void* A, const void* B, float s,
     return DORA_ERR_CUDA;
 
   // 1) B^T and (s c B)^T
+  note_launch();
   norm_bwd_prep_kernel<<<dim3(static_cast<unsigned>(cdiv(d_out, kPrepTile)), static_cast<unsigned>(cdiv(r, kPrepTile))),
                          256, 0, st>>>(static_cast<const __nv_bfloat16*>(B), d_n, n, s, static_cast<int>(d_out),
                                static_cast<int>(r), Bt, Bct);
@@ -1029,6 +1051,7 @@ int dora_factored_norm_bwd(const void* W, const void* A, const void* B, float s,
   ga.wait_limit = kWaitLimitCycles;
   ga.status = dev->status;
   const size_t gram_smem = kGramStages * kGramStageBytes + (2 * kGramStages + 1) * 8 + 16 + 1024;
+  note_launch();
   gram_tc_kernel<<<ga.n_ctas1 + L.nt * L.nt * ga.splits2, kNormThreads, gram_smem, st>>>(tmA, tmA, tmBct, tmBt, ga);
   if (launch_error()) return DORA_ERR_CUDA;
   {
@@ -1040,6 +1063,7 @@ int dora_factored_norm_bwd(const void* W, const void* A, const void* B, float s,
     const int g1 = static_cast<int>(std::max<long long>(1, std::min<long long>(cdiv(rr, 1024), 2 * dev->num_sms)));
     cfg.gridDim = dim3(static_cast<unsigned>(2 * g1));
     cfg.blockDim = dim3(256);
+    note_launch();
     if (cudaLaunchKernelEx(&cfg, gram_reduce_kernel, static_cast<const float*>(part), ga.splits, static_cast<int>(r), s,
                            sG, static_cast<int*>(nullptr), 0, g1, static_cast<const float*>(part2), ga.splits2, s,
                            s2H, 1) != cudaSuccess)
@@ -1085,6 +1109,7 @@ int dora_factored_norm_bwd(const void* W, const void* A, const void* B, float s,
   lb.wait_limit = kWaitLimitCycles;
   lb.status = dev->status;
   pcfg.gridDim = pair_grid(lb);
+  note_launch();
   if (cudaLaunchKernelEx(&pcfg, linear_pair_kernel<false, true>, tmW, tmAb, tmB, tmSG, lb) != cudaSuccess)
     return DORA_ERR_CUDA;
 
@@ -1108,6 +1133,7 @@ int dora_factored_norm_bwd(const void* W, const void* A, const void* B, float s,
   la.wait_limit = kWaitLimitCycles;
   la.status = dev->status;
   pcfg.gridDim = pair_grid(la);
+  note_launch();
   if (cudaLaunchKernelEx(&pcfg, linear_pair_kernel<true, true>, tmBct, tmWmn, tmH, tmAmn, la) != cudaSuccess)
     return DORA_ERR_CUDA;
   return launch_error();

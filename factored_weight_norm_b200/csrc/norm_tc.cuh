@@ -53,6 +53,7 @@ constexpr int kMaxChunkN = 512;       // TMEM columns
 constexpr int kMaxStages = 8;
 constexpr int kStatusTimeout = 5;     // == DORA_ERR_TIMEOUT
 constexpr int kFinOwners = 4;         // partial owners the finalizing warp loads together
+constexpr int kBAhead = 8;            // units before a segment's end at which its B rows are prefetched to L2
 
 struct NormArgs {
   int d_out, d_in, r;
@@ -172,6 +173,11 @@ struct UnitIter {
   __device__ __forceinline__ bool valid() const { return left > 0; }
   __device__ __forceinline__ bool seg_last(const NormArgs& a) const {
     return left == 1 || kb == a.kb_total - 1 || (len2 > 0 && left == len2 + 1);
+  }
+  // Units of this segment after the current one.
+  __device__ __forceinline__ int seg_rem(const NormArgs& a) const {
+    const int to_range_end = (len2 > 0 && left > len2) ? left - len2 - 1 : left - 1;
+    return min(a.kb_total - 1 - kb, to_range_end);
   }
   __device__ __forceinline__ void next(const NormArgs& a) {
     --left;
@@ -300,11 +306,15 @@ __global__ void __launch_bounds__(kNormTcThreads, 1)
     for (x.start(a, u_begin, u_end); x.valid() && ok; x.next(a)) {
       const int nboxes = (x.n_this + kBoxRows - 1) / kBoxRows;
       const bool ext = x.kb >= a.kb_main;
-      if (x.seg_first) {
-        // B's rows for this segment's epilogue: into L2 now, so that the ring
-        // loads of them at the segment end do not wait for HBM
-        const int nbox = (x.n_this + kBK - 1) / kBK;
-        for (int b = lane; b < nbox; b += 32) tma_prefetch_l2_2d(&tmB, x.c0 + b * kBK, x.mt * kBM);
+      {
+        // B's rows for this segment's epilogue: into L2 kBAhead units before
+        // the segment ends, so that the ring loads of them at its end do not
+        // wait for HBM (and the W stream has no time to evict them first)
+        const int rem = x.seg_rem(a);
+        if (rem == kBAhead || (x.seg_first && rem < kBAhead)) {
+          const int nbox = (x.n_this + kBK - 1) / kBK;
+          for (int b = lane; b < nbox; b += 32) tma_prefetch_l2_2d(&tmB, x.c0 + b * kBK, x.mt * kBM);
+        }
       }
       if (ext && !gram_ready) {
         grid_dep_wait();  // G' is written by the Gram kernels

@@ -78,6 +78,7 @@ SIGNATURES = {
     "dora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "dora_device_status": (ctypes.c_int, [_c_void_p]),
     "dora_num_sms": (ctypes.c_int, []),
+    "dora_launch_count": (ctypes.c_uint64, []),
     "dora_selftest_timeout": (ctypes.c_int, [_i64, _c_void_p]),
     "dora_factored_norm_batched_workspace_size": (_size, [_problems_p, ctypes.c_int, ctypes.c_int]),
     "dora_factored_norm_batched": (ctypes.c_int, [_problems_p, ctypes.c_int, ctypes.c_int, _c_void_p, _size, _c_void_p]),
@@ -212,6 +213,11 @@ def dora_compose_bwd_workspace_size(tokens: int, d_out: int) -> int:
 
 def dora_num_sms() -> int:
     return int(lib().dora_num_sms())
+
+
+def dora_launch_count() -> int:
+    """Kernels the library has launched in this process so far."""
+    return int(lib().dora_launch_count())
 
 
 def dora_device_status(stream=None) -> int:

@@ -318,6 +318,12 @@ DORA_API int dora_selftest_timeout(int64_t limit_cycles, void* stream);
  * device (the grid is a multiple of this count).  Returns 0 when no device. */
 DORA_API int dora_num_sms(void);
 
+/* Kernels this library has launched in this process, on any device and
+ * stream (a host-side count, incremented as each launch is enqueued; a
+ * launch that fails still counts).  For a caller that counts the library's
+ * GPU work over a region: read it before and after. */
+DORA_API uint64_t dora_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif

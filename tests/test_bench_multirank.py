@@ -46,7 +46,8 @@ def _rank_main(rank, world, port, out_dir):
         if rank == 0:
             wl = bench.WL.HEADLINE
             res = dict(t_total=got[0], t_norm=got[1], t_fwd=got[2], t_bwd=got[3], clocks=None, status=0, wl=wl,
-                       e2e=dict(t_norm=2 * got[1], t_fwd=2 * got[2], t_bwd=2 * got[3], h2d=10, d2h=20, steps=5))
+                       e2e=dict(t_norm=2 * got[1], t_fwd=2 * got[2], t_bwd=2 * got[3], h2d=10, d2h=20, steps=5),
+                       launches=28, flushed=False)
 
             class Args:
                 steps, warmup = 7, 3
@@ -100,6 +101,44 @@ def test_line_counts_both_replicas(two_ranks):
     assert line["norm"]["frac"] == pytest.approx(F / 0.75 / 1e12 / 1000.0)
     assert line["roofline"]["kernel"] == "norm" and line["roofline"]["traffic"] is None
     assert line["e2e"]["value"] == pytest.approx(2 * F / 1.5 / 1e12)
+    assert line["gpu_launches"] == 28 and line["dtype"] == "bf16"
+    assert line["config"]["l2"].startswith("no flush")
+
+
+def _line_for(bench, wl, traffic, flushed=False):
+    res = dict(t_total=1.0, t_norm=1e-4, t_fwd=1e-4, t_bwd=1e-4, clocks=None, status=0, wl=wl,
+               e2e=dict(t_norm=2e-4, t_fwd=2e-4, t_bwd=2e-4, h2d=10, d2h=20, steps=5), launches=4, flushed=flushed)
+
+    class Args:
+        steps, warmup = 1, 3
+
+    return bench.build_line(Args, res, 1, {"bf16_tflops": 1000.0, "hbm_gbs": 5000.0}, "test", traffic, None)
+
+
+def test_traffic_is_taken_only_for_its_own_workload():
+    """A traffic row counts only for the workload it was captured on: the
+    headline's rows give nothing to the 4096 module, whose line says null."""
+    bench = _bench()
+    traffic = {("norm", "bf16_8192_r384"): 150e6, ("compose_fwd", "bf16_8192_r384_T8192"): 410e6,
+               ("compose_bwd", "bf16_8192_r384_T8192"): 680e6}
+    head = _line_for(bench, bench.WL.HEADLINE, traffic)
+    assert [k["traffic"] for k in head["rooflines"]] == [150e6, 410e6, 680e6]
+    other = _line_for(bench, bench.WL.SINGLE_4096, traffic)
+    assert [k["traffic"] for k in other["rooflines"]] == [None, None, None]
+    # a headline run with another token count has no compose row either
+    t4096 = _line_for(bench, bench.WL.HEADLINE.with_(tokens=4096), traffic)
+    assert [k["traffic"] for k in t4096["rooflines"]] == [150e6, None, None]
+
+
+def test_dtype_and_l2_follow_the_workload():
+    bench = _bench()
+    tiny = bench.WL.TINY_F32
+    assert bench.step_bytes(tiny) < 2 * bench.L2_BYTES  # the tiny step is flushed before every step
+    line = _line_for(bench, tiny, {}, flushed=True)
+    assert line["dtype"] == "f32"
+    assert line["config"]["l2"].startswith("flushed before every step")
+    # fp32 moves four bytes an element
+    assert line["norm"]["bytes"] == bench.norm_bytes(tiny.d_out, tiny.d_in, tiny.r, 4)
 
 
 def test_reference_arm_runs_on_rank_zero_only(two_ranks):
