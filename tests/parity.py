@@ -89,3 +89,45 @@ def near_unity_check(y_gpu, y_exact, base, max_midpoint_fraction=1e-3):
     frac = float(rescued.sum()) / max(1, y_gpu.size)
     assert frac <= max_midpoint_fraction, f"midpoint clause used on {frac:.2e} of elements"
     return frac
+
+
+# ---------------------------------------------------- norm-gradient bounds
+# The attached-norm backward computes dB = s c (W A^T + B (sG)^T) and
+# dA = (s c B)^T W + (s^2 H) A with c = d_n / n, G = A A^T, H = (c B)^T B; it
+# rounds (s c B), sG and s^2 H to bf16 and accumulates every product in fp32.
+# Rounding x to bf16 moves it by at most u |x| (u = 2^-8, eight significant
+# bits); an fp32 sum of K terms is off by at most K 2^-24 times the sum of
+# the terms' magnitudes; each rounded intermediate's error is carried through
+# the product that uses it by the magnitudes of the other factor.
+U_BF16 = 2.0 ** -8   # unit roundoff of bf16 (8 significant bits)
+E_F32 = 2.0 ** -24   # unit roundoff of fp32
+
+
+def grad_bounds(W, A, B, s, n, d_n, rows=None, cols=None):
+    """First-order bounds (fp64 arrays) on |gpu - exact| for dA [r, d_in] and
+    dB [d_out, r] (only dA's `cols` and dB's `rows` when given), from the
+    arithmetic described above."""
+    W, A, B = (np.asarray(x, dtype=np.float64) for x in (W, A, B))
+    n, d_n = np.asarray(n, dtype=np.float64), np.asarray(d_n, dtype=np.float64)
+    d_out, d_in = W.shape
+    r = A.shape[0]
+    u, e = U_BF16, E_F32
+    c = d_n / n
+    aA, aB = np.abs(A), np.abs(B)
+    # ---- dB rows: s c_i (sum_k W_ik A_jk + sum_l B_il (sG)_lj), one fp32 sum over d_in + r
+    Wr = W if rows is None else W[rows]
+    Br, cr = (B, c) if rows is None else (B[rows], c[rows])
+    sG = s * (A @ A.T)
+    sG_err = u * np.abs(sG) + d_in * e * abs(s) * (aA @ aA.T)  # its fp32 sum, then bf16
+    termW = np.abs(Wr) @ aA.T
+    termG = np.abs(Br) @ np.abs(sG)
+    eB = np.abs(s * cr)[:, None] * ((d_in + r) * e * (termW + termG) + np.abs(Br) @ sG_err + e * (termW + termG))
+    # ---- dA columns: sum_i (s c_i B_ij) W_ik + sum_l (s^2 H)_jl A_lk, one fp32 sum over d_out + r
+    Wc, Ac = (W, A) if cols is None else (W[:, cols], A[:, cols])
+    scB = (s * c)[:, None] * B
+    s2H = s * (scB.T @ B)
+    s2H_err = u * np.abs(s2H) + (u + d_out * e) * abs(s) * (np.abs(scB).T @ aB)  # (s c B) in bf16, fp32 sum, bf16
+    termB = np.abs(scB).T @ np.abs(Wc)
+    termH = np.abs(s2H) @ np.abs(Ac)
+    eA = u * termB + s2H_err @ np.abs(Ac) + (d_out + r) * e * (termB + termH)
+    return eA, eB

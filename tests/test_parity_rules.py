@@ -4,6 +4,7 @@ g = m / n to bf16 first (the cancellation the Scaling DoRA abstract warns
 about for the near-unity regime)."""
 
 import numpy as np
+import pytest
 import torch
 
 import oracle
@@ -71,3 +72,69 @@ def test_norm_tolerances():
         except AssertionError:
             continue
         raise AssertionError("norm tolerance not enforced")
+
+
+# ------------------------------------------- the norm-gradient error model
+def _bf16(x):
+    return torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16).double().numpy()
+
+
+def _emulated_norm_bwd(W, A, B, s, n, d_n, plant=None):
+    """The backward's arithmetic on the CPU: (s c B), sG and s^2 H rounded to
+    bf16, every product summed in fp32 (float32 matmuls), outputs fp32."""
+    f32 = np.float32
+    c = (d_n.astype(f32) / n.astype(f32)).astype(np.float64)
+    sG = _bf16((s * (A.astype(f32) @ A.astype(f32).T)).astype(np.float64))
+    scB = _bf16((s * c)[:, None] * B)
+    s2H = _bf16((s * (scB.astype(f32).T @ B.astype(f32))).astype(np.float64))
+    if plant == "drop_gram":
+        sG = np.zeros_like(sG)
+    if plant == "H_scale":
+        s2H = s2H / s
+    K1 = np.concatenate([W, B], axis=1).astype(f32)
+    N1 = np.concatenate([A, sG], axis=1).astype(f32)
+    dB = (s * c)[:, None] * (K1 @ N1.T).astype(np.float64)
+    dA = (scB.astype(f32).T @ W.astype(f32)).astype(np.float64) + (s2H.astype(f32) @ A.astype(f32)).astype(np.float64)
+    if plant == "transpose_B":
+        dB = dB[:, ::-1].copy()
+    return dA.astype(np.float32).astype(np.float64), dB.astype(np.float32).astype(np.float64)
+
+
+@pytest.mark.parametrize("shape,s", [((96, 160, 32), 0.5), ((64, 512, 48), -2.0), ((200, 96, 16), 1.25)])
+def test_grad_bound_covers_the_kernels_arithmetic(shape, s):
+    """An fp32/bf16 emulation of the backward's arithmetic stays within twice
+    the per-element bound of the exact (oracle) gradients."""
+    d_out, d_in, r = shape
+    rng = np.random.default_rng(7)
+    W = _bf16(rng.standard_normal((d_out, d_in)) * 0.02)
+    A = _bf16(rng.uniform(-1, 1, (r, d_in)) / np.sqrt(d_in))
+    B = _bf16(rng.standard_normal((d_out, r)) * 0.01)
+    n = np.linalg.norm(W + s * (B @ A), axis=1).astype(np.float32).astype(np.float64)
+    d_n = rng.standard_normal(d_out)
+    rA, rB = oracle.norm_backward(W, A, B, s, n, d_n)
+    gA, gB = _emulated_norm_bwd(W, A, B, s, n, d_n)
+    eA, eB = P.grad_bounds(W, A, B, s, n, d_n)
+    assert (np.abs(gA - rA) <= 2 * eA + 1e-30).all()
+    assert (np.abs(gB - rB) <= 2 * eB + 1e-30).all()
+    # the bound stays a small fraction of the gradients themselves (dA's sums
+    # over d_out cancel, so its worst-case bound is the looser one): not vacuous
+    assert np.median(eA / np.maximum(np.abs(rA), 1e-300)) < 0.1
+    assert np.median(eB / np.maximum(np.abs(rB), 1e-300)) < 0.02
+
+
+@pytest.mark.parametrize("plant", ["drop_gram", "H_scale", "transpose_B"])
+def test_grad_bound_rejects_a_planted_mistake(plant):
+    """A dropped Gram term, a wrong power of s on H or permuted dB columns
+    leave the bound somewhere."""
+    d_out, d_in, r, s = 128, 96, 32, 0.5
+    rng = np.random.default_rng(11)
+    W = _bf16(rng.standard_normal((d_out, d_in)) * 0.02)
+    A = _bf16(rng.uniform(-1, 1, (r, d_in)) / np.sqrt(d_in))
+    B = _bf16(rng.standard_normal((d_out, r)) * 0.05)
+    n = np.linalg.norm(W + s * (B @ A), axis=1).astype(np.float32).astype(np.float64)
+    d_n = rng.standard_normal(d_out)
+    rA, rB = oracle.norm_backward(W, A, B, s, n, d_n)
+    gA, gB = _emulated_norm_bwd(W, A, B, s, n, d_n, plant=plant)
+    eA, eB = P.grad_bounds(W, A, B, s, n, d_n)
+    outside = (np.abs(gA - rA) > 2 * eA).any() or (np.abs(gB - rB) > 2 * eB).any()
+    assert outside, plant
