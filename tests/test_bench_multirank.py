@@ -136,7 +136,7 @@ def test_dtype_and_l2_follow_the_workload():
     assert bench.step_bytes(tiny) < 2 * bench.L2_BYTES  # the tiny step is flushed before every step
     line = _line_for(bench, tiny, {}, flushed=True)
     assert line["dtype"] == "f32"
-    assert line["config"]["l2"].startswith("flushed before every step")
+    assert line["config"]["l2"].startswith("L2 cleaned before every step")
     # fp32 moves four bytes an element
     assert line["norm"]["bytes"] == bench.norm_bytes(tiny.d_out, tiny.d_in, tiny.r, 4)
 
