@@ -128,30 +128,30 @@ __global__ void __launch_bounds__(256, 3) compose_fwd_kernel(const T* __restrict
   }
   const long long row0 = blockIdx.y * rows_per_cta;
   const long long row1 = min(tokens, row0 + rows_per_cta);
-  long long row = row0;
   constexpr int U = 4;
-  for (; row + U <= row1; row += U) {
-    float b[U][VEC], l[U][VEC];
+  // U rows per pass, their loads issued together; the last pass predicates
+  // the rows past row1 (one memory round trip for the leftover rows too)
+  using Raw = typename VecIO<T, VEC>::Raw;
+  for (long long row = row0; row < row1; row += U) {
+    Raw rb[U], rl[U];  // packed until used: fewer registers with U rows in flight
 #pragma unroll
     for (int k = 0; k < U; ++k) {
-      VecIO<T, VEC>::load(base + (row + k) * d_out + col, b[k]);
-      VecIO<T, VEC>::load(lora + (row + k) * d_out + col, l[k]);
+      if (row + k < row1) {
+        rb[k] = VecIO<T, VEC>::raw(base + (row + k) * d_out + col);
+        rl[k] = VecIO<T, VEC>::raw(lora + (row + k) * d_out + col);
+      }
     }
 #pragma unroll
     for (int k = 0; k < U; ++k) {
-      float o[VEC];
+      if (row + k < row1) {
+        float b[VEC], l[VEC], o[VEC];
+        VecIO<T, VEC>::unpack(rb[k], b);
+        VecIO<T, VEC>::unpack(rl[k], l);
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) o[e] = b[k][e] + fmaf(delta[e], b[k][e] - bb[e], gs[e] * l[k][e]);
-      VecIO<T, VEC>::store(y + (row + k) * d_out + col, o);
+        for (int e = 0; e < VEC; ++e) o[e] = b[e] + fmaf(delta[e], b[e] - bb[e], gs[e] * l[e]);
+        VecIO<T, VEC>::store(y + (row + k) * d_out + col, o);
+      }
     }
-  }
-  for (; row < row1; ++row) {
-    float b[VEC], l[VEC], o[VEC];
-    VecIO<T, VEC>::load(base + row * d_out + col, b);
-    VecIO<T, VEC>::load(lora + row * d_out + col, l);
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) o[e] = b[e] + fmaf(delta[e], b[e] - bb[e], gs[e] * l[e]);
-    VecIO<T, VEC>::store(y + row * d_out + col, o);
   }
 }
 
