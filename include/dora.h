@@ -71,7 +71,9 @@ typedef enum {
 } dora_status;
 
 /* Bytes of workspace dora_factored_norm needs for this shape (0 never means
- * "no workspace" for valid shapes; returns 0 for invalid shapes). */
+ * "no workspace" for valid shapes; returns 0 for invalid shapes): the
+ * O(d_out r + r^2) intermediates of the factored norm (Scaling DoRA, Abstract),
+ * here (s/2) A A^T in bf16 and per-row partial sums, never O(d_out d_in). */
 DORA_API size_t dora_factored_norm_workspace_size(int64_t d_out, int64_t d_in, int64_t r, dora_dtype dt);
 
 /* Factored row norm of W + s B A (Scaling DoRA, Abstract: "base, cross, and
@@ -167,10 +169,16 @@ DORA_API int dora_compose_fwd_bias(const void* base_out, const void* lora_out, c
                                    const float* n, float s, int64_t tokens, int64_t d_out, dora_dtype dt, void* y,
                                    void* stream);
 
-/* Bytes of workspace dora_compose_bwd needs (column partial sums). */
+/* Bytes of workspace dora_compose_bwd needs: per-chunk partial sums of d_m
+ * over tokens, O(d_out), independent of tokens beyond a bounded chunk count
+ * (the single-pass backward of Scaling DoRA, Abstract, keeps no
+ * [tokens, d_out] intermediate). */
 DORA_API size_t dora_compose_bwd_workspace_size(int64_t tokens, int64_t d_out);
 
-/* Backward of dora_compose_fwd with n held constant (the norm is detached):
+/* Backward of dora_compose_fwd with n held constant (the norm is detached;
+ * Scaling DoRA, Abstract: the fused compose "for both forward and gradient
+ * computation"; DoRA summary page, Method: the gradient of the magnitude m and
+ * of the direction's low-rank factors):
  *
  *   d_base = g * dy,   d_lora = s * g * dy,
  *   d_m_i  = (sum_t dy[t,i] * (base[t,i] + s * lora[t,i])) / n_i
@@ -235,7 +243,8 @@ DORA_API int dora_compose_bwd_noalloc_bias(const void* dy, const void* base_out,
 
 /* Bytes of workspace dora_factored_norm_bwd needs: O(r^2 + r d_out), no
  * d_out x d_in term (the Gram partial tiles, s G and s^2 H in bf16, and two
- * [r, d_out] bf16 copies of B). */
+ * [r, d_out] bf16 copies of B), as the factored norm's intermediates are
+ * (Scaling DoRA, Abstract). */
 DORA_API size_t dora_factored_norm_bwd_workspace_size(int64_t d_out, int64_t d_in, int64_t r);
 
 /* Gradients of the row norms n_i = ||W_i + s B_i A|| into A and B, for
@@ -267,7 +276,8 @@ DORA_API int dora_factored_norm_bwd(const void* W, const void* A, const void* B,
                                     float* dA, float* dB, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Bytes of workspace dora_fused_linear_fwd needs: the [tokens, r] bf16
- * intermediate P = s * x A^T (at least 256). */
+ * intermediate P = s * x A^T (at least 256), the LoRA branch's down
+ * projection (DoRA summary page, Method: the low-rank update B A). */
 DORA_API size_t dora_fused_linear_fwd_workspace_size(int64_t tokens, int64_t r);
 
 /* The DoRA linear forward with the compose fused into the GEMMs that produce
