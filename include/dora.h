@@ -76,8 +76,9 @@ typedef enum {
  * here (s/2) A A^T in bf16 and per-row partial sums, never O(d_out d_in). */
 DORA_API size_t dora_factored_norm_workspace_size(int64_t d_out, int64_t d_in, int64_t r, dora_dtype dt);
 
-/* Factored row norm of W + s B A (Scaling DoRA, Abstract: "base, cross, and
- * Gram terms computable through O(d_out r + r^2) intermediates"):
+/* Factored row norm of W + s B A (Scaling DoRA, Abstract: the squared norm
+ * splits into a base, a cross and a Gram term, which need only
+ * O(d_out r + r^2) intermediates):
  *
  *   n_i = sqrt(max(||W_i||^2 + 2 s <B_i, (W A^T)_i> + s^2 B_i (A A^T) B_i^T, 0))
  *
@@ -124,7 +125,7 @@ typedef struct {
 DORA_API size_t dora_factored_norm_batched_workspace_size(const dora_norm_problem* problems, int count, dora_dtype dt);
 
 /* The factored row norms of `count` adapted modules at once (Scaling DoRA,
- * Abstract: models carry "hundreds of adapted modules"), each computing
+ * Abstract: a model carries hundreds of adapted modules), each computing
  * exactly what dora_factored_norm computes for it.  `problems` is a host
  * array, read during the call only.  Modules with bf16 weights and
  * 16 <= r <= 512 share two launches: every 128 x 128 tile of every module's
@@ -176,8 +177,8 @@ DORA_API int dora_compose_fwd_bias(const void* base_out, const void* lora_out, c
 DORA_API size_t dora_compose_bwd_workspace_size(int64_t tokens, int64_t d_out);
 
 /* Backward of dora_compose_fwd with n held constant (the norm is detached;
- * Scaling DoRA, Abstract: the fused compose "for both forward and gradient
- * computation"; DoRA summary page, Method: the gradient of the magnitude m and
+ * Scaling DoRA, Abstract: the fused compose serves the forward pass and the
+ * gradients; DoRA summary page, Method: the gradient of the magnitude m and
  * of the direction's low-rank factors):
  *
  *   d_base = g * dy,   d_lora = s * g * dy,
@@ -248,8 +249,8 @@ DORA_API int dora_compose_bwd_noalloc_bias(const void* dy, const void* base_out,
 DORA_API size_t dora_factored_norm_bwd_workspace_size(int64_t d_out, int64_t d_in, int64_t r);
 
 /* Gradients of the row norms n_i = ||W_i + s B_i A|| into A and B, for
- * training with the norm kept attached (Scaling DoRA, Abstract: the factored
- * norm's "gradient computation"; the default DoRA backward, dora_compose_bwd,
+ * training with the norm kept attached (Scaling DoRA, Abstract: gradients
+ * through the factored norm; the default DoRA backward, dora_compose_bwd,
  * holds n constant).  With c = d_n / n and never forming B A:
  *
  *   dB = s c * (W A^T + s B G),            G = A A^T

@@ -105,7 +105,7 @@ def dense_adapted_weight(W, A, B, s) -> np.ndarray:
 def row_norm(W, A, B, s) -> np.ndarray:
     """``n_i = ||W_i + s * B_i A||_2`` for every output channel i.
 
-    Scaling DoRA, Abstract ("the row-wise norm of W + sBA"); DoRA summary
+    Scaling DoRA, Abstract (the norm is taken over each row of W + sBA); DoRA summary
     page, Method (per-output-channel vector norm of the adapted weight).
     """
     Wp = dense_adapted_weight(W, A, B, s)
@@ -211,7 +211,7 @@ def norm_backward(W, A, B, s, n, d_n):
     """Gradients of the row norms ``n_i = ||W_i + s B_i A||`` w.r.t. ``A`` and ``B``.
 
     For the training variant that keeps the norm attached (Scaling DoRA,
-    Abstract, "gradient computation"; the DoRA summary page's Method defines
+    Abstract, gradients through the norm; the DoRA summary page's Method defines
     the norm of the adapted weight ``V = W + sBA``).  ``d_n`` is the upstream
     gradient of the loss w.r.t. ``n`` (for the DoRA compose it is
     ``-(m / n) * d_m``).  Chain rule on the dense definition: ``dn_i/dV_i =
