@@ -14,18 +14,24 @@
 // [d_out, r] product V never leaves TMEM.
 //
 // Kernels (one stream, chained with programmatic dependent launch):
-//   gram_tc_kernel     G = A A^T as 128x128 tiles split over K (fp32 partials)
-//   gram_reduce_kernel sums the K splits in fixed order, writes bf16 G'
+//   gram_cluster_kernel (gram_cluster.cuh) G' = (s/2) A A^T from clusters of
+//                      K splits on a few SMs; also zeroes the tile counters
 //   norm_tc_kernel     persistent stream-K GEMM over (M tile, N chunk, K
-//                      block) units; each CTA owns a contiguous unit range and
-//                      starts streaming W before the Gram kernels finish (it
-//                      only waits for them before its first K-extension block).
-//                      Two warps sum ||W_i||^2 from the shared-memory W
-//                      stages; at each segment end B's rows arrive through
-//                      the same TMA ring and four epilogue warps dot them
-//                      with V_i read from TMEM; one fp32 partial per (row,
-//                      segment); the last warp to finish an M tile sums its
-//                      partials in fixed order and writes n = sqrt(max(., 0)).
+//                      block) units in weighted contiguous ranges (shorter
+//                      for the CTAs that start behind the Gram clusters); a
+//                      range that crosses a tile boundary is walked from that
+//                      boundary on, so its K-extension blocks (the only reads
+//                      of G') come last and the GEMM seldom waits for the
+//                      Gram launch.  Two warps sum ||W_i||^2 from the
+//                      shared-memory W stages; at each segment end B's rows
+//                      arrive through the same TMA ring and four epilogue
+//                      warps dot them with V_i read from TMEM; one fp32
+//                      partial per (row, segment); the last warp to finish an
+//                      M tile sums its partials in fixed order and writes
+//                      n = sqrt(max(., 0)).
+// gram_tc_kernel and gram_reduce_kernel below (split-K Gram tiles and their
+// fixed-order reduction) serve the attached-norm backward's two Gram
+// products.
 #pragma once
 
 #include "sm100_ptx.cuh"
