@@ -69,39 +69,9 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, l
   return __all_sync(0xffffffffu, ok);
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // Orders this thread's generic-proxy accesses (all state spaces) with its
 // later async-proxy accesses, e.g. TMA loads of data other threads wrote.
 __device__ __forceinline__ void fence_proxy_async_all() { asm volatile("fence.proxy.async;" ::: "memory"); }
-
-__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-// Spins until *p >= target (acquire), for at most `limit` SM cycles.  The
-// poll interval backs off to about a microsecond so that many CTAs polling
-// one counter do not crowd out the atomic updates they are waiting for.
-__device__ __forceinline__ bool spin_until_geq(const int* p, int target, long long limit) {
-  if (ld_acquire_gpu(p) >= target) return true;
-  const long long t0 = clock64();
-  unsigned ns = 64;
-  while (ld_acquire_gpu(p) < target) {
-    __nanosleep(ns);
-    if (ns < 1024) ns <<= 1;
-    if (clock64() - t0 > limit) return false;
-  }
-  return true;
-}
-
-// Named barrier over `count` threads (a multiple of 32) of this CTA.
-__device__ __forceinline__ void named_bar_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
 
 // ------------------------------------------------- programmatic dependent launch
 // Waits until every grid this one depends on (launched earlier on the stream
