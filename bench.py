@@ -258,10 +258,13 @@ def run_ours(args, rank, world, local_rank):
     clocks = sampler.stop() if sampler else None
     status = D.dora_device_status()
 
-    t_norm = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps * 1e-3
-    t_fwd = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps * 1e-3
-    t_bwd = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps * 1e-3
+    per_step = {k: [e[i].elapsed_time(e[i + 1]) * 1e-3 for e in evs] for i, k in enumerate(("norm", "fwd", "bwd"))}
+    t_norm = sum(per_step["norm"]) / args.steps
+    t_fwd = sum(per_step["fwd"]) / args.steps
+    t_bwd = sum(per_step["bwd"]) / args.steps
     t_total = (t_norm + t_fwd + t_bwd) * args.steps  # the cleans between steps are not the step's
+    spread = {k: {"median_us": statistics.median(v) * 1e6, "min_us": min(v) * 1e6, "max_us": max(v) * 1e6}
+              for k, v in per_step.items()}
 
     # the same steps back to back without the clean: the norm then also
     # writes back what the previous compose backward left dirty in L2
@@ -298,7 +301,7 @@ def run_ours(args, rank, world, local_rank):
     fused = idle_then(lambda: run_fused_linear_context(D, dev, wl, W, A, B, m, n)) if bf16_ctx else None
     return dict(t_total=t_total, t_norm=t_norm, t_fwd=t_fwd, t_bwd=t_bwd, clocks=clocks, status=status, e2e=e2e,
                 wl=wl, dense=dense, batched=batched, fused=fused, norm_bwd=norm_bwd, launches=launches,
-                flushed=True, unflushed=dict(t_total=u_total, t_norm=u_norm, t_fwd=u_fwd, t_bwd=u_bwd))
+                flushed=True, unflushed=dict(t_total=u_total, t_norm=u_norm, t_fwd=u_fwd, t_bwd=u_bwd), spread=spread)
 
 
 def run_dense_comparator(D, dev, W, A, B, s, ws_n, reps=10):
@@ -669,6 +672,7 @@ def build_line(args, res, N, peaks, peak_src, traffic, cpu):
         },
         "norm": {"tflops": F / res["t_norm"] / 1e12, "frac": rl[0]["frac"], "bound": norm_bound,
                  "time_us": res["t_norm"] * 1e6, "flops": F, "bytes": Bn},
+        "step_time_spread": res.get("spread"),
         "roofline": {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
                     | {"kernel": dominant["kernel"], "peak_source": dominant["peak_source"]},
         "rooflines": rl,
