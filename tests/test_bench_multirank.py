@@ -130,6 +130,26 @@ def test_traffic_is_taken_only_for_its_own_workload():
     assert [k["traffic"] for k in t4096["rooflines"]] == [150e6, None, None]
 
 
+def test_line_carries_the_step_spread_and_the_unflushed_pass():
+    bench = _bench()
+    wl = bench.WL.HEADLINE
+    res = dict(t_total=2.0, t_norm=1e-4, t_fwd=2e-4, t_bwd=3e-4, clocks=None, status=0, wl=wl,
+               e2e=dict(t_norm=2e-4, t_fwd=2e-4, t_bwd=2e-4, h2d=10, d2h=20, steps=5), launches=4, flushed=True,
+               unflushed=dict(t_total=2.2, t_norm=1.2e-4, t_fwd=2e-4, t_bwd=3e-4),
+               spread={"norm": {"median_us": 99.0, "min_us": 98.0, "max_us": 120.0}})
+
+    class Args:
+        steps, warmup = 10, 3
+
+    line = bench.build_line(Args, res, 1, {"bf16_tflops": 1000.0, "hbm_gbs": 5000.0}, "test", {}, None)
+    assert line["step_time_spread"]["norm"]["max_us"] == 120.0
+    F = bench.norm_flops(wl.d_out, wl.d_in, wl.r)
+    u = line["steps_without_clean"]
+    assert u["norm"]["time_us"] == pytest.approx(120.0)
+    assert u["norm"]["tflops"] == pytest.approx(F / 1.2e-4 / 1e12)
+    assert u["ms_per_step"] == pytest.approx(2.2 / 10 * 1e3)
+
+
 def test_dtype_and_l2_follow_the_workload():
     bench = _bench()
     tiny = bench.WL.TINY_F32
