@@ -378,12 +378,14 @@ int norm_bf16(const void* W, const void* A, const void* B, int64_t d_out, int64_
     // 0.43 us per K block of its split, plus about 5 us to sum and mirror
     // off-diagonal tiles; a GEMM unit about 0.18 us plus 0.01 us per KB of its
     // ring stage.  A late CTA that ends early costs the grid a little; one
-    // that ends late costs the whole gap, so the delay is taken 10% long.
+    // that ends late costs the whole gap, so the delay is taken 10% long,
+    // 25% for Gram phases past 20 us, which the linear model underestimates
+    // (r = 768 at 8192 x 8192: 111.7 against 115.7 us with 10%).
     const int gram_sms = std::min(dev->num_sms, up_tiles * splits);
     const int late = grid > gram_sms ? gram_sms : 0;
     const double gram_us = 3.0 + 0.43 * static_cast<double>(cdiv(p.kb_main, splits)) + (nt > 1 ? 5.0 : 1.0);
     const double unit_us = 0.18 + 0.01 * (static_cast<double>(na.stage_bytes) / 1024.0);
-    const double delay = 1.1 * gram_us / unit_us;
+    const double delay = (gram_us > 20.0 ? 1.25 : 1.1) * gram_us / unit_us;
     const double f = (static_cast<double>(p.units) + late * delay) / grid;
     na.early = grid - late;
     na.w_early = std::max<long long>(1, std::llround(16.0 * f));
